@@ -1,0 +1,170 @@
+"""Pins for the oracle's prefix GEMV, routing, prefix selection and MoE layer."""
+import itertools
+import math
+
+import numpy as np
+import pytest
+
+from conftest import read_golden
+
+
+def _dequant(oracle_mod, codes, scales, cb, G, b, bf16=False):
+    lv = oracle_mod.level(cb.astype(np.float32), b)
+    s = np.repeat(scales, G, axis=1)
+    if bf16:
+        v = (s * lv[codes >> (8 - b)]).astype(np.float32)  # float product, then bf16 rounding
+        u = v.view(np.uint32).astype(np.uint64)
+        u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
+        return u.astype(np.uint32).view(np.float32).astype(np.float64)
+    return s.astype(np.float64) * lv[codes >> (8 - b)].astype(np.float64)
+
+
+@pytest.mark.parametrize("b", range(1, 9))
+def test_gemv_against_numpy_dequant_matmul(oracle_mod, synth_mod, b):
+    w = synth_mod.expert_weights(5, 0, 0, 0, 128, 256)
+    scales, codes = oracle_mod.quantize(w, 64)
+    cb = oracle_mod.tree_codebook_f32()
+    x = synth_mod.activation_f32(5, 0, 0, 256).astype(np.float64)
+    y = oracle_mod.gemv(codes, scales, cb, 64, b, x)
+    ref = _dequant(oracle_mod, codes, scales, cb, 64, b) @ x
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-15)
+    yb = oracle_mod.gemv(codes, scales, cb, 64, b, x, bf16_weights=True)
+    refb = _dequant(oracle_mod, codes, scales, cb, 64, b, bf16=True) @ x
+    np.testing.assert_allclose(yb, refb, rtol=1e-12, atol=1e-15)
+
+
+def test_gemv_unit_vectors(oracle_mod):
+    """x = e_k returns column k of the dequantised matrix: scale * C[b][code >> (8-b)]."""
+    rng = np.random.default_rng(1)
+    codes = rng.integers(0, 256, size=(16, 128), dtype=np.uint8)
+    scales = rng.uniform(0.5, 2.0, size=(16, 2)).astype(np.float32)
+    cb = oracle_mod.tree_codebook_f32()
+    for k in (0, 63, 64, 127):
+        x = np.zeros(128)
+        x[k] = 1.0
+        for b in (1, 3, 8):
+            y = oracle_mod.gemv(codes, scales, cb, 64, b, x)
+            lv = oracle_mod.level(cb, b)
+            expect = scales[:, k // 64].astype(np.float64) * lv[codes[:, k] >> (8 - b)]
+            np.testing.assert_array_equal(y, expect)
+
+
+def test_route_hand_examples(oracle_mod):
+    logits = np.array([[0.5, 2.0, 2.0, -1.0, 1.0, 2.0],
+                       [0.0, 0.0, 0.0, 0.0, 0.0, 0.0]], dtype=np.float32)
+    ids, w = oracle_mod.route(logits, 3)
+    np.testing.assert_array_equal(ids[0], [1, 2, 5])      # ties go to the lower id
+    np.testing.assert_array_equal(ids[1], [0, 1, 2])
+    np.testing.assert_allclose(w[0], [1 / 3] * 3, rtol=1e-7)
+    np.testing.assert_allclose(w[1], [1 / 3] * 3, rtol=1e-7)
+
+
+def test_route_against_sort_and_softmax(oracle_mod, synth_mod):
+    E, k = 512, 10
+    logits = np.stack([synth_mod.router_logits(9, t, 0, E) for t in range(64)])
+    ids, w = oracle_mod.route(logits, k)
+    for t in range(64):
+        order = sorted(range(E), key=lambda e: (-float(logits[t, e]), e))[:k]
+        np.testing.assert_array_equal(ids[t], order)
+        sel = logits[t, order].astype(np.float64)
+        ref = np.exp(sel - sel.max()) / np.exp(sel - sel.max()).sum()
+        np.testing.assert_allclose(w[t], ref, rtol=1e-7)
+        assert abs(float(w[t].astype(np.float64).sum()) - 1.0) < 1e-6
+
+
+def _objective(w, s, b):
+    return sum(float(wi) ** 2 * float(si) ** 2 * 4.0 ** (-int(bi)) for wi, si, bi in zip(w, s, b))
+
+
+@pytest.mark.parametrize("k", [1, 2, 3, 4])
+def test_select_is_brute_force_optimum(oracle_mod, k):
+    """Greedy on w^2 s^2 4^-b equals the exhaustive minimum under sum b = B (cue 29)."""
+    rng = np.random.default_rng(k)
+    for trial in range(40):
+        w = rng.dirichlet(np.ones(k)).astype(np.float32)[None, :]
+        ids = np.arange(k, dtype=np.int32)[None, :]
+        sens = np.exp(0.5 * rng.standard_normal(k)).astype(np.float32)
+        avg = float(rng.choice([1.0, 1.5, 2.5, 3.25, 5.0, 8.0]))
+        B = oracle_mod.budget(k, avg)
+        d = oracle_mod.select(w, ids, sens, avg)[0]
+        assert int(d.sum()) == B
+        best = math.inf
+        for cand in itertools.product(range(1, 9), repeat=k):
+            if sum(cand) == B:
+                best = min(best, _objective(w[0], sens, cand))
+        got = _objective(w[0], sens, d)
+        assert got == pytest.approx(best, rel=1e-12)
+
+
+def test_select_equals_offset_rule(oracle_mod, synth_mod):
+    """b_i = clamp(ceil(c + log2(w_i s_i / geomean)), 1, 8), c set so that mean b = 2.5."""
+    E, k = 512, 10
+    sens = synth_mod.sensitivities(2, 0, E)
+    logits = np.stack([synth_mod.router_logits(2, t, 0, E) for t in range(200)])
+    ids, w = oracle_mod.route(logits, k)
+    depth = oracle_mod.select(w, ids, sens, 2.5)
+    for t in range(200):
+        v = (w[t] * sens[ids[t]]).astype(np.float32).astype(np.float64)
+        lg = np.log2(v) - np.log2(v).mean()
+        # breakpoints of the step function c -> sum clamp(ceil(c + lg), 1, 8)
+        bps = sorted({n - x for x in lg for n in range(-20, 30)})
+        ok = None
+        for lo, hi in zip(bps[:-1], bps[1:]):
+            c = 0.5 * (lo + hi)
+            b = np.clip(np.ceil(c + lg), 1, 8)
+            if b.sum() == 25:
+                ok = b
+                break
+        assert ok is not None
+        np.testing.assert_array_equal(depth[t], ok.astype(np.uint8))
+        assert depth[t].mean() == 2.5
+
+
+def test_select_budget_and_candidates(oracle_mod):
+    rows = read_golden("allocator_candidates.txt")
+    k, first, last, cand = map(int, rows[0])
+    assert k * (last - first) == cand          # 10 experts x 7 upgrades = 70 (cue 29)
+    assert oracle_mod.budget(10, 2.5) == 25
+    assert oracle_mod.budget(8, 2.5) == 20
+    assert oracle_mod.budget(10, 0.1) == 10     # clamped to one bit each
+    assert oracle_mod.budget(10, 9.0) == 80     # clamped to eight bits each
+    w = np.full((1, 10), 0.1, np.float32)
+    ids = np.arange(10, dtype=np.int32)[None, :]
+    d = oracle_mod.select(w, ids, np.ones(10, np.float32), 8.0)
+    assert np.all(d == 8)
+    d = oracle_mod.select(w, ids, np.ones(10, np.float32), 2.5)
+    # all priorities equal: upgrades cycle through the slots in order
+    np.testing.assert_array_equal(d[0], [3, 3, 3, 3, 3, 2, 2, 2, 2, 2])
+
+
+def test_moe_layer_against_numpy(oracle_mod, synth_mod):
+    E, k, H, I, G, T = 8, 3, 256, 128, 64, 3
+    cb = oracle_mod.tree_codebook_f32()
+    experts = {}
+    deq = {}
+    for e in range(E):
+        codes, scales = [], []
+        for m, (n, kk) in enumerate(((I, H), (I, H), (H, I))):
+            s, c = oracle_mod.quantize(synth_mod.expert_weights(4, 0, e, m, n, kk), G)
+            codes.append(c)
+            scales.append(s)
+        experts[e] = oracle_mod.Expert(codes, scales, [cb, cb, cb])
+    logits = np.stack([synth_mod.router_logits(4, t, 0, E) for t in range(T)])
+    ids, w = oracle_mod.route(logits, k)
+    sens = synth_mod.sensitivities(4, 0, E)
+    depth = oracle_mod.select(w, ids, sens, 2.5)
+    x = np.stack([synth_mod.bf16_to_f32(synth_mod.activation_bf16(4, t, 0, H)) for t in range(T)])
+    y = oracle_mod.moe_layer(experts, E, H, I, G, ids, w, depth, x.astype(np.float64))
+    for t in range(T):
+        ref = np.zeros(H)
+        for i in range(k):
+            e, b = int(ids[t, i]), int(depth[t, i])
+            ex = experts[e]
+            Wg = _dequant(oracle_mod, ex.codes[0], ex.scales[0], cb, G, b)
+            Wu = _dequant(oracle_mod, ex.codes[1], ex.scales[1], cb, G, b)
+            Wd = _dequant(oracle_mod, ex.codes[2], ex.scales[2], cb, G, b)
+            g = Wg @ x[t]
+            u = Wu @ x[t]
+            h = g / (1 + np.exp(-g)) * u
+            ref += float(w[t, i]) * (Wd @ h)
+        np.testing.assert_allclose(y[t], ref, rtol=1e-10, atol=1e-13)
