@@ -1,0 +1,412 @@
+"""Benchmark: batch-1 MoE-layer decode on bitplane prefixes (one B200 per rank).
+
+Workload (N=1): a seeded synthetic MoE layer of the pages' model shape -- 512
+experts, top-10, hidden 4096, expert intermediate 1024, SwiGLU, group-128
+scales, all 8 planes of every expert resident in HBM (6.4 GB) -- decoding
+batch-1 tokens at an average of 2.5 bits per routed expert. One step = the
+whole hot path for one fresh token: route (top-10 + softmax), prefix
+selection, grouping, gate/up prefix GEMV + SwiGLU, down prefix GEMV and the
+weighted combine, all on the device.
+
+Multi-GPU: replicas only (one independent layer replica per rank, weak
+scaling); the path has no exchange step.
+
+--impl reference times the CPU oracle (the plain single-threaded C
+implementation) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer decode tokens/s; achieved HBM GB/s on bitplane bytes vs B200 peak"
+WORKLOAD = "moe_layer_e512_top10_h4096_i1024_g128_avg2.5_batch1"
+E, K_TOP, H, I, G, AVG = 512, 10, 4096, 1024, 128, 2.5
+SEED = 2026
+N_TOKENS = 1024
+PLANE_BYTES = H * I // 8                    # one plane of one matrix
+SCALE_BYTES = 3 * (H * I // G) * 4          # scales of one expert (3 matrices)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=64)
+    ap.add_argument("--impl", default="pmoe", choices=["pmoe", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=400)
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+def traffic_from_profiles():
+    """Per-launch DRAM bytes of the expert kernels from the committed ncu summary, if current."""
+    p = os.path.join(ROOT, "profiles", "expert_kernels_traffic.txt")
+    try:
+        with open(p) as f:
+            for line in f:
+                if line.startswith("traffic_bytes_per_token:"):
+                    return float(line.split(":")[1])
+    except OSError:
+        pass
+    return None
+
+
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- oracle legs
+
+def oracle_token_setup(seed, token_ids):
+    """Quantise (oracle) the experts the given tokens select; returns per-token inputs."""
+    import numpy as np
+
+    import oracle
+    import synth
+    sens = synth.sensitivities(seed, 0, E)
+    cb = oracle.tree_codebook_f32()
+    toks = []
+    experts = {}
+    for t in token_ids:
+        logits = synth.router_logits(seed, t, 0, E)[None, :]
+        xb = synth.activation_bf16(seed, t, 0, H)[None, :]
+        ids, _ = oracle.route(logits, K_TOP)
+        for e in ids[0]:
+            e = int(e)
+            if e not in experts:
+                codes, scales = [], []
+                for m, (n, kk) in enumerate(((I, H), (I, H), (H, I))):
+                    s, c = oracle.quantize(synth.expert_weights(seed, 0, e, m, n, kk), G)
+                    codes.append(c)
+                    scales.append(s)
+                experts[e] = oracle.Expert(codes, scales, [cb] * 3)
+        toks.append((logits, synth.bf16_to_f32(xb).astype(np.float64)))
+    return sens, experts, toks
+
+
+def oracle_token(sens, experts, logits, x64):
+    import oracle
+    ids, w = oracle.route(logits, K_TOP)
+    dep = oracle.select(w, ids, sens, AVG)
+    need = {int(e): experts[int(e)] for e in ids[0]}
+    return oracle.moe_layer(need, E, H, I, G, ids, w, dep, x64)
+
+
+def cpu_baseline(seed):
+    """The oracle, as it stands, on one full token of the workload (single thread)."""
+    sens, experts, toks = oracle_token_setup(seed, [0])
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        oracle_token(sens, experts, *toks[0])
+        n += 1
+        if time.perf_counter() - t0 > 8.0 or n >= 8:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} x one full batch-1 token (route, select, 10 experts x gate/up/down at "
+                      f"the selected depths, SwiGLU, combine) in double, experts pre-quantised"}
+
+
+def reference_arm(args):
+    """The base contract's reference arm for this build: the CPU oracle, bounded samples."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np
+
+    import oracle
+    sens, experts, toks = oracle_token_setup(SEED, [0])
+    logits, x64 = toks[0]
+    ids, w = oracle.route(logits, K_TOP)
+    dep = oracle.select(w, ids, sens, AVG)
+    # one step = a slice of rows of the token's expert matrices at the selected depths;
+    # sized so warmup + steps take about a minute.
+    mats = [(int(ids[0, i]), m, int(dep[0, i])) for i in range(K_TOP) for m in range(3)]
+    weights_per_token = 3 * H * I * K_TOP
+    probe_rows = 64
+    ex = experts[mats[0][0]]
+    t0 = time.perf_counter()
+    oracle.gemv(ex.codes[0][:probe_rows], ex.scales[0][:probe_rows], ex.cbs[0], G, mats[0][2], x64[0])
+    rate = probe_rows * H / max(time.perf_counter() - t0, 1e-6)        # weights/s
+    budget = 60.0 / max(args.steps + args.warmup, 1)
+    rows = max(16, min(I, int(rate * budget / H) // 16 * 16))
+    h_vec = np.zeros(I)
+    done_w = 0
+
+    def step(i):
+        nonlocal done_w
+        e, m, b = mats[i % len(mats)]
+        ex = experts[e]
+        r0 = ((i // len(mats)) * rows) % (ex.codes[m].shape[0] - rows + 1)
+        x = x64[0] if m < 2 else h_vec
+        oracle.gemv(ex.codes[m][r0:r0 + rows], ex.scales[m][r0:r0 + rows], ex.cbs[m], G, b, x)
+        done_w += rows * ex.codes[m].shape[1]
+
+    for i in range(args.warmup):
+        step(i)
+    done_w = 0
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    dt = time.perf_counter() - t0
+    tok = done_w / weights_per_token
+    val = tok / dt
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / max(args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD},
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": f"per step: {rows} rows of one selected expert matrix at its "
+                                       f"selected depth (dequantise-then-matvec in double); tokens "
+                                       f"counted as decoded weights / {weights_per_token}"},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import __graft_entry__
+    __graft_entry__.build()
+    import bitplane_mixed_precision_b200 as pm
+    import synth
+    from bitplane_mixed_precision_b200.store import ResidentLayer
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+
+    def fill(e, m, w):
+        synth.expert_weights_device(SEED, 0, e, m, w.numel(), w.data_ptr(), stream.cuda_stream)
+
+    R = ResidentLayer(E, H, I, G, fill, device=dev)
+    sens = torch.from_numpy(synth.sensitivities(SEED, 0, E)).to(dev)
+    tok0 = rank * 1_000_000
+    logits_h = np.stack([synth.router_logits(SEED, tok0 + t, 0, E) for t in range(N_TOKENS)])
+    x_h = np.stack([synth.activation_bf16(SEED, tok0 + t, 0, H) for t in range(N_TOKENS)])
+    logits = torch.from_numpy(logits_h).to(dev)
+    x = torch.from_numpy(x_h.view(np.int16)).to(dev)
+    T = 1
+    ws_bytes = pm.layer_workspace_bytes(T, K_TOP, E, H, I)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    y = torch.empty(N_TOKENS, H, dtype=torch.float32, device=dev)
+    ids = torch.empty(N_TOKENS, K_TOP, dtype=torch.int32, device=dev)
+    wts = torch.empty(N_TOKENS, K_TOP, dtype=torch.float32, device=dev)
+    dep = torch.empty(N_TOKENS, K_TOP, dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+
+    def step(i, st):
+        j = i % N_TOKENS
+        pm.moe_decode_step(R.layer, logits[j], sens, x[j], T, K_TOP, AVG, y[j], ids[j], wts[j], dep[j],
+                           ws, ws_bytes, st)
+
+    kernels_per_step = 7  # route+select, group, prep, gate/up, h-prep, down, combine
+
+    # warm-up (eager)
+    for i in range(args.warmup):
+        step(i, stream)
+    torch.cuda.synchronize()
+
+    # live kernel timing of the expert kernels, L2 flushed before each token
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(N_TOKENS)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(N_TOKENS)]
+    n_prof = min(N_TOKENS, 512)
+    for i in range(n_prof):
+        flush.fill_(i & 0xFF)
+        pm.profile_events(ev0[i], ev1[i])
+        step(i, stream)
+    pm.profile_events(None, None)
+    torch.cuda.synchronize()
+    kdur = [ev0[i].elapsed_time(ev1[i]) * 1e-3 for i in range(n_prof)]
+    dep_h = dep[:n_prof].cpu().numpy().astype(np.int64)
+    plane_bytes = dep_h.sum(axis=1) * 3 * PLANE_BYTES
+    alg_bytes = plane_bytes + K_TOP * SCALE_BYTES + H * 2 + H * 4
+    achieved = float(alg_bytes.sum() / sum(kdur)) / 1e9
+    bitplane_gbs = float(plane_bytes.sum() / sum(kdur)) / 1e9
+
+    # graph-captured timed steps
+    gsize = min(args.steps, N_TOKENS)
+    graphs = []
+    cap = torch.cuda.Stream(dev)
+    for n_in_graph in ([gsize] + ([args.steps % gsize] if args.steps % gsize else [])):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            for i in range(n_in_graph):
+                step(i, cap)
+        graphs.append((g, n_in_graph))
+    full_reps = args.steps // gsize
+    for g, _ in graphs:
+        g.replay()
+    torch.cuda.synchronize()
+
+    pr = torch.cuda.get_device_properties(dev)
+    clocks = ClockSampler(f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0")
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.2)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for _ in range(full_reps):
+        graphs[0][0].replay()
+    if len(graphs) > 1:
+        graphs[1][0].replay()
+    t_stop.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    elapsed = t_start.elapsed_time(t_stop) * 1e-3
+    if world > 1:
+        tt = torch.tensor([elapsed], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        elapsed = float(tt.item())
+        dist.barrier()
+    value = args.steps * world / elapsed
+
+    # end to end through the C ABI with host buffers (pinned), one token per step
+    ne = min(args.e2e_steps, N_TOKENS)
+    lg_pin = torch.from_numpy(logits_h[:ne]).pin_memory()
+    x_pin = torch.from_numpy(x_h[:ne].view(np.int16)).pin_memory()
+    y_pin = torch.empty(ne, H, dtype=torch.float32).pin_memory()
+    lg_d = torch.empty(E, dtype=torch.float32, device=dev)
+    x_d = torch.empty(H, dtype=torch.int16, device=dev)
+    y_d = torch.empty(H, dtype=torch.float32, device=dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for i in range(ne):
+        lg_d.copy_(lg_pin[i], non_blocking=True)
+        x_d.copy_(x_pin[i], non_blocking=True)
+        pm.moe_decode_step(R.layer, lg_d, sens, x_d, T, K_TOP, AVG, y_d, None, None, None, ws, ws_bytes,
+                           stream)
+        y_pin[i].copy_(y_d, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_t = e0.elapsed_time(e1) * 1e-3
+    if world > 1:
+        tt = torch.tensor([e2e_t], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_t = float(tt.item())
+    e2e = {"value": ne * world / e2e_t, "unit": "tokens/s", "h2d_bytes_per_step": E * 4 + H * 2,
+           "d2h_bytes_per_step": H * 4}
+
+    for g, _ in graphs:
+        del g
+    graphs.clear()
+
+    if rank == 0:
+        pk, pk_kind = peaks()
+        peak = float(pk["hbm_gbs"])
+        traffic = traffic_from_profiles()
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = cpu_baseline(SEED)
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": elapsed * 1e3 / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "s8 mma / s32 acc / f32",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "experts": E, "top_k": K_TOP, "hidden": H, "inter": I,
+                       "group": G, "avg_bits": AVG, "batch": 1, "tokens_distinct": N_TOKENS,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (6.4 GB of resident planes), fresh token per step; "
+                             "kernel timing with L2 flushed before each token"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "kernel": "expert kernels (gate/up+SwiGLU, h fragments, down)",
+                         "peak_kind": f"{pk_kind} hbm_gbs"},
+            "bitplane_gbs": bitplane_gbs, "bitplane_frac_of_8000": bitplane_gbs / 8000.0,
+            "expert_kernels_us": 1e6 * sum(kdur) / len(kdur),
+            "mean_bits": float(dep_h.mean()),
+            "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": kernels_per_step * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

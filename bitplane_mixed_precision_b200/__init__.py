@@ -1,0 +1,182 @@
+"""Python binding of libpmoe (bitplane-prefix MoE expert execution on B200).
+
+Argument marshalling only: every function forwards to the C ABI declared in
+``include/pmoe.h`` under the same name (without the ``pmoe_`` prefix) and
+raises :class:`PmoeError` on a non-OK status. Pointers may be given as torch
+tensors, numpy arrays or integers. There is no fallback: importing this
+package fails if ``libpmoe.so`` has not been built (``build.build()``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpmoe.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libpmoe.so is missing at {LIB_PATH}; build it with "
+                      "`python -m bitplane_mixed_precision_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+P = ctypes.c_void_p
+i32, i64, f32, sz = ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+
+
+class Matrix(ctypes.Structure):
+    """pmoe_matrix: one stored expert matrix (device pointers)."""
+    _fields_ = [("planes", P), ("plane_stride_words", i64), ("scales", P), ("codebook", P),
+                ("N", i32), ("K", i32), ("G", i32)]
+
+
+class Layer(ctypes.Structure):
+    """pmoe_layer: one MoE layer's experts in a plane-slot pool (device pointers)."""
+    _fields_ = [("E", i32), ("H", i32), ("I", i32), ("G", i32), ("pool", P), ("slot_words", i64),
+                ("slot_of", P), ("scales", P), ("codebooks", P)]
+
+
+_SIGS = {
+    "pmoe_status_string": ([i32], ctypes.c_char_p),
+    "pmoe_last_cuda_error": ([], i32),
+    "pmoe_version": ([], i32),
+    "pmoe_tree_codebook": ([P], i32),
+    "pmoe_quantize": ([P, i32, i32, i32, P, P, P], i32),
+    "pmoe_pack_bitplanes": ([P, i32, i32, i32, P, i64, i32, P], i32),
+    "pmoe_extract_prefix": ([P, i64, i32, i32, i32, P, P], i32),
+    "pmoe_route": ([P, i32, i32, i32, P, P, P], i32),
+    "pmoe_select_prefix": ([P, P, P, i32, i32, f32, P, i32, P], i32),
+    "pmoe_expert_gemv": ([ctypes.POINTER(Matrix), i32, P, i32, P, P], i32),
+    "pmoe_layer_workspace_bytes": ([i32, i32, i32, i32, i32], sz),
+    "pmoe_moe_layer_fwd": ([ctypes.POINTER(Layer), P, P, P, P, i32, i32, P, P, sz, P], i32),
+    "pmoe_moe_decode_step": ([ctypes.POINTER(Layer), P, P, P, i32, i32, f32, P, P, P, P, P, sz, P],
+                             i32),
+    "pmoe_profile_events": ([P, P], i32),
+    "pmoe_materialise_workspace_bytes": ([i32, i32, i32, i32, i32], sz),
+    "pmoe_materialise_layer_fwd": ([ctypes.POINTER(Layer), P, P, P, P, i32, i32, P, P, sz, P], i32),
+}
+
+for _name, (_args, _res) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = _res
+
+
+def exported_symbols():
+    """Names the binding resolves in libpmoe.so (each must exist)."""
+    return sorted(_SIGS)
+
+
+class PmoeError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        msg = _lib.pmoe_status_string(code).decode()
+        if code == 2:
+            msg += f" (cudaError {_lib.pmoe_last_cuda_error()})"
+        super().__init__(f"{fn}: {msg}")
+        self.code = code
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if hasattr(x, "data_ptr"):
+        return x.data_ptr()
+    if hasattr(x, "ctypes"):
+        return x.ctypes.data
+    raise TypeError(f"cannot take a pointer of {type(x)}")
+
+
+def _stream(s):
+    if s is None:
+        return None
+    if hasattr(s, "cuda_stream"):
+        return s.cuda_stream
+    return int(s)
+
+
+def _check(fn, rc):
+    if rc != 0:
+        raise PmoeError(fn, rc)
+
+
+def version() -> int:
+    return _lib.pmoe_version()
+
+
+def tree_codebook(out) -> None:
+    _check("pmoe_tree_codebook", _lib.pmoe_tree_codebook(_ptr(out)))
+
+
+def quantize(w, N, K, G, scales, codes, stream=None) -> None:
+    _check("pmoe_quantize", _lib.pmoe_quantize(_ptr(w), N, K, G, _ptr(scales), _ptr(codes), _stream(stream)))
+
+
+def pack_bitplanes(codes, N, K, depth, planes, plane_stride_words, on_device=True, stream=None) -> None:
+    _check("pmoe_pack_bitplanes", _lib.pmoe_pack_bitplanes(_ptr(codes), N, K, depth, _ptr(planes),
+                                                           plane_stride_words, int(on_device),
+                                                           _stream(stream)))
+
+
+def extract_prefix(planes, plane_stride_words, N, K, b, idx, stream=None) -> None:
+    _check("pmoe_extract_prefix", _lib.pmoe_extract_prefix(_ptr(planes), plane_stride_words, N, K, b,
+                                                           _ptr(idx), _stream(stream)))
+
+
+def route(logits, T, E, k, ids, w, stream=None) -> None:
+    _check("pmoe_route", _lib.pmoe_route(_ptr(logits), T, E, k, _ptr(ids), _ptr(w), _stream(stream)))
+
+
+def select_prefix(w, ids, sens, T, k, avg_bits, depth, on_device=True, stream=None) -> None:
+    _check("pmoe_select_prefix", _lib.pmoe_select_prefix(_ptr(w), _ptr(ids), _ptr(sens), T, k, avg_bits,
+                                                         _ptr(depth), int(on_device), _stream(stream)))
+
+
+def make_matrix(planes, plane_stride_words, scales, codebook, N, K, G) -> Matrix:
+    return Matrix(_ptr(planes), plane_stride_words, _ptr(scales), _ptr(codebook), N, K, G)
+
+
+def expert_gemv(m: Matrix, b, x, x_is_bf16, y, stream=None) -> None:
+    _check("pmoe_expert_gemv", _lib.pmoe_expert_gemv(ctypes.byref(m), b, _ptr(x), int(x_is_bf16), _ptr(y),
+                                                     _stream(stream)))
+
+
+def make_layer(E, H, I, G, pool, slot_words, slot_of, scales, codebooks) -> Layer:
+    return Layer(E, H, I, G, _ptr(pool), slot_words, _ptr(slot_of), _ptr(scales), _ptr(codebooks))
+
+
+def layer_workspace_bytes(T, k, E, H, I) -> int:
+    return _lib.pmoe_layer_workspace_bytes(T, k, E, H, I)
+
+
+def moe_layer_fwd(L: Layer, x, ids, w, depth, T, k, y, ws, ws_bytes, stream=None) -> None:
+    _check("pmoe_moe_layer_fwd", _lib.pmoe_moe_layer_fwd(ctypes.byref(L), _ptr(x), _ptr(ids), _ptr(w),
+                                                         _ptr(depth), T, k, _ptr(y), _ptr(ws), ws_bytes,
+                                                         _stream(stream)))
+
+
+def moe_decode_step(L: Layer, logits, sens, x, T, k, avg_bits, y, ids_out, w_out, depth_out, ws,
+                    ws_bytes, stream=None) -> None:
+    _check("pmoe_moe_decode_step", _lib.pmoe_moe_decode_step(
+        ctypes.byref(L), _ptr(logits), _ptr(sens), _ptr(x), T, k, avg_bits, _ptr(y), _ptr(ids_out),
+        _ptr(w_out), _ptr(depth_out), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def profile_events(start, stop) -> None:
+    """start/stop: torch.cuda.Event (or raw cudaEvent_t ints); None, None disables."""
+    def h(e):
+        if e is None:
+            return None
+        return e.cuda_event if hasattr(e, "cuda_event") else int(e)
+    _check("pmoe_profile_events", _lib.pmoe_profile_events(h(start), h(stop)))
+
+
+def materialise_workspace_bytes(T, k, E, H, I) -> int:
+    return _lib.pmoe_materialise_workspace_bytes(T, k, E, H, I)
+
+
+def materialise_layer_fwd(L: Layer, x, ids, w, depth, T, k, y, ws, ws_bytes, stream=None) -> None:
+    _check("pmoe_materialise_layer_fwd", _lib.pmoe_materialise_layer_fwd(
+        ctypes.byref(L), _ptr(x), _ptr(ids), _ptr(w), _ptr(depth), T, k, _ptr(y), _ptr(ws), ws_bytes,
+        _stream(stream)))

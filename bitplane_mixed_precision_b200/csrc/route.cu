@@ -1,0 +1,116 @@
+// Routing (top-k + softmax, PagedMoE transcript cue 4) and prefix selection
+// (greedy bit allocation on w^2 * E_e(b), transcript cues 29-31).
+#include "common.h"
+#include "dev.cuh"
+#include "route.cuh"
+
+namespace pmoe {
+
+// ---------------------------------------------------------------- host selection
+
+// Greedy: all experts start at 1 bit; B-k times the largest w*s*2^-b (ties to
+// the lower slot, 8-bit experts skipped) gets one more bit.
+static void select_host(const float *w, const int32_t *ids, const float *sens, int T, int k,
+                        float avg_bits, uint8_t *depth)
+{
+    const int B = select_budget(k, avg_bits);
+    float v[32];
+    int b[32];
+    for (int t = 0; t < T; ++t) {
+        for (int i = 0; i < k; ++i) {
+            v[i] = w[t * k + i] * sens[ids[t * k + i]];
+            b[i] = 1;
+        }
+        for (int step = k; step < B; ++step) {
+            int best = -1;
+            float bp = 0.0f;
+            for (int i = 0; i < k; ++i) {
+                if (b[i] >= 8)
+                    continue;
+                const float pr = ldexpf(v[i], -b[i]);
+                if (best < 0 || pr > bp) {
+                    best = i;
+                    bp = pr;
+                }
+            }
+            if (best < 0)
+                break;
+            b[best] += 1;
+        }
+        for (int i = 0; i < k; ++i)
+            depth[t * k + i] = (uint8_t)b[i];
+    }
+}
+
+// ---------------------------------------------------------------- device kernels
+
+// One warp per token; see route.cuh for the two device functions.
+__global__ void route_kernel(const float *__restrict__ logits, int T, int E, int k,
+                             int32_t *__restrict__ ids, float *__restrict__ w)
+{
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (warp >= T)
+        return;
+    int id;
+    float wt;
+    dev::route_token(logits + (int64_t)warp * E, E, k, id, wt);
+    const int lane = threadIdx.x & 31;
+    if (lane < k) {
+        ids[warp * k + lane] = id;
+        w[warp * k + lane] = wt;
+    }
+}
+
+__global__ void select_kernel(const float *__restrict__ w, const int32_t *__restrict__ ids,
+                              const float *__restrict__ sens, int T, int k, int B,
+                              uint8_t *__restrict__ depth)
+{
+    __shared__ float prio[4][7 * 32];
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (warp >= T)
+        return;
+    const int lane = threadIdx.x & 31;
+    float v = 0.0f;
+    if (lane < k)
+        v = __fmul_rn(w[warp * k + lane], sens[ids[warp * k + lane]]);
+    const int b = dev::select_token(v, k, B, prio[(threadIdx.x >> 5) & 3]);
+    if (lane < k)
+        depth[warp * k + lane] = (uint8_t)b;
+}
+
+} // namespace pmoe
+
+using namespace pmoe;
+
+extern "C" {
+
+pmoe_status pmoe_route(const float *logits, int T, int E, int k, int32_t *ids, float *w,
+                       pmoe_stream stream)
+{
+    if (!logits || !ids || !w || T < 0 || k < 1 || k > 32 || E < k || E > 4096)
+        return PMOE_ERR_INVALID_ARG;
+    if (T == 0)
+        return PMOE_OK;
+    const int blocks = (T + 3) / 4;
+    route_kernel<<<blocks, 128, 0, (cudaStream_t)stream>>>(logits, T, E, k, ids, w);
+    return launch_status();
+}
+
+pmoe_status pmoe_select_prefix(const float *w, const int32_t *ids, const float *sens, int T, int k,
+                               float avg_bits, uint8_t *depth, int on_device, pmoe_stream stream)
+{
+    if (!w || !ids || !sens || !depth || T < 0 || k < 1 || k > 32 || !(avg_bits == avg_bits))
+        return PMOE_ERR_INVALID_ARG;
+    if (T == 0)
+        return PMOE_OK;
+    if (!on_device) {
+        select_host(w, ids, sens, T, k, avg_bits, depth);
+        return PMOE_OK;
+    }
+    const int B = select_budget(k, avg_bits);
+    const int blocks = (T + 3) / 4;
+    select_kernel<<<blocks, 128, 0, (cudaStream_t)stream>>>(w, ids, sens, T, k, B, depth);
+    return launch_status();
+}
+
+} // extern "C"

@@ -1,0 +1,88 @@
+// Warp-level routing and prefix selection for one token.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace pmoe {
+namespace dev {
+
+// Order-preserving map of float to uint32 (larger float -> larger key, > 0).
+__device__ __forceinline__ uint32_t ord_key(float f)
+{
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Top-k of l[0..E) (ties to the lower id), descending, and softmax over the k
+// (PagedMoE transcript cue 4: k experts, weights summing to one). Executed by
+// a full warp; lane s < k receives slot s. Lane c holds ids c, c+32, ...
+__device__ __forceinline__ void route_token(const float *__restrict__ l, int E, int k, int &id_out,
+                                            float &w_out)
+{
+    const int lane = threadIdx.x & 31;
+    uint32_t taken[4] = {0u, 0u, 0u, 0u}; // E <= 4096: 128 ids per lane
+    auto local_best = [&](uint32_t &bk, int &bj) {
+        bk = 0u;
+        bj = -1;
+        for (int j = 0; lane + 32 * j < E; ++j) {
+            if ((taken[j >> 5] >> (j & 31)) & 1u)
+                continue;
+            const uint32_t key = ord_key(__ldg(l + lane + 32 * j));
+            if (key > bk) {
+                bk = key;
+                bj = j;
+            }
+        }
+    };
+    uint32_t bk;
+    int bj;
+    local_best(bk, bj);
+    int my_id = 0;
+    float my_l = 0.0f;
+    for (int s = 0; s < k; ++s) {
+        const uint32_t gmax = __reduce_max_sync(0xffffffffu, bk);
+        const unsigned cand = (bj >= 0 && bk == gmax) ? (unsigned)(lane + 32 * bj) : 0x7fffffffu;
+        const unsigned win = __reduce_min_sync(0xffffffffu, cand);
+        if (lane == s) {
+            my_id = (int)win;
+            my_l = __ldg(l + win);
+        }
+        if (lane == (int)(win & 31u)) {
+            const int j = (int)(win >> 5);
+            taken[j >> 5] |= 1u << (j & 31);
+            local_best(bk, bj);
+        }
+    }
+    const double l0 = (double)__shfl_sync(0xffffffffu, my_l, 0);
+    const double e = (lane < k) ? exp((double)my_l - l0) : 0.0;
+    double sum = 0.0;
+    for (int s = 0; s < k; ++s)
+        sum = __dadd_rn(sum, __shfl_sync(0xffffffffu, e, s));
+    id_out = my_id;
+    w_out = (lane < k) ? __double2float_rn(__ddiv_rn(e, sum)) : 0.0f;
+}
+
+// Greedy prefix selection for one token (transcript cue 29): lane i < k holds
+// v_i = w_i * s_{e_i}; B - k rounds grant one bit to the largest v_i * 2^-b_i
+// (exact ldexp; ties to the lower slot; 8-bit slots skipped). Returns b_i.
+__device__ __forceinline__ int select_token(float v, int k, int B, float * /*unused scratch*/)
+{
+    const int lane = threadIdx.x & 31;
+    int b = 1;
+    for (int step = k; step < B; ++step) {
+        const bool ok = lane < k && b < 8;
+        const uint32_t key = ok ? __float_as_uint(ldexpf(v, -b)) : 0u;
+        const uint32_t gmax = __reduce_max_sync(0xffffffffu, ok ? key : 0u);
+        const unsigned tied = __ballot_sync(0xffffffffu, ok && key == gmax);
+        if (tied == 0u)
+            break;
+        if (lane == __ffs(tied) - 1)
+            b += 1;
+    }
+    return b;
+}
+
+} // namespace dev
+} // namespace pmoe

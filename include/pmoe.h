@@ -1,0 +1,248 @@
+/*
+ * pmoe.h — C ABI of libpmoe: direct execution of bitplane prefixes of routed
+ * MoE experts on NVIDIA B200 (sm_100a).
+ *
+ * Sources (web pages on PagedMoE, cited by page and section):
+ *   [T#n] "PagedMoE: Cross-Precision Expert Caching for SSD-Resident MoE
+ *         Inference", podcast transcript, subtitle cue n.
+ *   [A]   "PagedMoE: Cross-Precision Expert Caching for Token-Level Dynamic
+ *         Precision in SSD-Resident MoE Inference", arxivlens page, Abstract
+ *         and Methodology.
+ *
+ * Conventions for every entry point:
+ *   - Pointers are plain host or device pointers, as stated per argument.
+ *     All memory is owned by the caller; no entry point frees or keeps a
+ *     pointer after it returns, except the cache object (pmoe_cache_*),
+ *     which keeps the device pool and page-table pointers given at creation.
+ *   - Calls that take a stream are asynchronous on it. Argument errors that
+ *     the host can see are returned before anything is enqueued, and then
+ *     nothing has been written.
+ *   - No entry point allocates device memory. Scratch is passed in by the
+ *     caller (workspace arguments) with the size given by the matching
+ *     *_workspace_bytes query.
+ *   - Return value: PMOE_OK or an error code below; pmoe_status_string()
+ *     names it. PMOE_ERR_CUDA means a CUDA call (launch or copy) failed;
+ *     pmoe_last_cuda_error() returns its cudaError_t value.
+ *
+ * Stored format of one expert matrix W (N rows x K columns) [T#19-#27, A]:
+ *   - codebook: 510 float32, the binary tree of a 256-entry sorted codebook;
+ *     depth d (1..8) node i at offset (1<<d)-2+i; truncating an 8-bit index
+ *     to its top b bits names its depth-b ancestor [T#21].
+ *   - scales: float32 [N][K/G], one per row and group of G columns.
+ *   - planes: 8 bitplanes of the 8-bit indices, MSB first: plane p holds bit
+ *     (7-p) of every index, so a depth-b read touches planes 0..b-1 only
+ *     [T#25]. Each plane is N*K/32 uint32 words; weight (n,k) of plane p is
+ *       tile = (n/16)*(K/128) + k/128, rr = n%16, kk = k%128,
+ *       g = rr%8, u = rr/8, s = kk/32, half = (kk%32)/16, t = (kk%16)/4,
+ *       i = kk%4, j = 4*half + i, L = 4*g + t, q = 2*s + u, h = q/4, r = q%4,
+ *       word = tile*64 + 2*L + h, bit = (4*j + p + r) mod 32.
+ *     (16x128 tiles; inside a tile lane L of a warp owns words 2L, 2L+1, and
+ *     the bit order lets a lane assemble 4-bit prefix indices with one AND
+ *     per plane and one rotate.) N % 16 == 0 and K % 128 == 0.
+ *   - The depth-b value of weight (n,k) is scales[n][k/G] * C[b][code>>(8-b)].
+ */
+#ifndef PMOE_H
+#define PMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PMOE_API __attribute__((visibility("default")))
+#else
+#define PMOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *pmoe_stream; /* a cudaStream_t; NULL = legacy default stream */
+typedef struct CUevent_st *pmoe_event;   /* a cudaEvent_t */
+
+typedef enum {
+    PMOE_OK = 0,
+    PMOE_ERR_INVALID_ARG = 1,  /* null pointer, bad size, shape or alignment */
+    PMOE_ERR_CUDA = 2,         /* a CUDA runtime call failed */
+    PMOE_ERR_OUT_OF_SLOTS = 3, /* the prefix cache cannot hold the request */
+    PMOE_ERR_BUDGET = 4,       /* infeasible bit budget */
+    PMOE_ERR_WORKSPACE = 5,    /* workspace too small */
+    PMOE_ERR_TIMEOUT = 6,      /* a bounded device wait ran out (see pmoe_moe_layer_fwd) */
+    PMOE_ERR_UNSUPPORTED = 7   /* shape or option this build does not handle */
+} pmoe_status;
+
+PMOE_API const char *pmoe_status_string(pmoe_status s);
+PMOE_API int pmoe_last_cuda_error(void);
+PMOE_API int pmoe_version(void);
+
+/* ------------------------------------------------------------------ */
+/* Format                                                              */
+/* ------------------------------------------------------------------ */
+
+/*
+ * pmoe_tree_codebook [T#19, T#21]: the tree codebook of N(0,1) values cut into
+ * 256 equiprobable bins: depth-d node i = conditional mean of N(0,1) on the
+ * quantile interval [i/2^d, (i+1)/2^d) (children have equal mass, so each
+ * parent is the mean of its children). Host only, synchronous.
+ *   codebook: host float[510], written. Returns PMOE_ERR_INVALID_ARG if NULL.
+ */
+PMOE_API pmoe_status pmoe_tree_codebook(float *codebook);
+
+/*
+ * pmoe_quantize: per-group scale and 8-bit index of every weight for the
+ * Gaussian tree codebook. scale = population std (double, sequential sum,
+ * rounded to float; 0 -> 1) of the G weights of a row group; index = number
+ * of thresholds Phi^-1(i/256), i = 1..255, at or below w/scale (double).
+ *   w: device float [N*K] row-major. scales: device float [N*(K/G)].
+ *   codes: device uint8 [N*K]. G divides K; N, K > 0.
+ */
+PMOE_API pmoe_status pmoe_quantize(const float *w, int N, int K, int G, float *scales, uint8_t *codes,
+                          pmoe_stream stream);
+
+/*
+ * pmoe_pack_bitplanes [T#25, A]: writes planes 0..depth-1 of the codes in the
+ * layout above. Plane p starts at planes + p*plane_stride_words
+ * (plane_stride_words >= N*K/32; it lets a caller pack straight into a slot
+ * pool). on_device = 1: codes and planes are device pointers, a warp-ballot
+ * kernel runs on the stream; 0: host pointers, synchronous host loop.
+ *   N % 16 == 0, K % 128 == 0, 1 <= depth <= 8.
+ */
+PMOE_API pmoe_status pmoe_pack_bitplanes(const uint8_t *codes, int N, int K, int depth, uint32_t *planes,
+                                int64_t plane_stride_words, int on_device, pmoe_stream stream);
+
+/*
+ * pmoe_extract_prefix [T#21, T#25]: reads planes 0..b-1 the way the GEMV
+ * kernels do and writes the b-bit prefix index code>>(8-b) of every weight.
+ * Device pointers. idx: device uint8 [N*K] row-major. 1 <= b <= 8.
+ */
+PMOE_API pmoe_status pmoe_extract_prefix(const uint32_t *planes, int64_t plane_stride_words, int N, int K,
+                                int b, uint8_t *idx, pmoe_stream stream);
+
+/* ------------------------------------------------------------------ */
+/* Routing and prefix selection                                        */
+/* ------------------------------------------------------------------ */
+
+/*
+ * pmoe_route [T#4]: per token, the k largest logits (ties to the lower expert
+ * id) in descending order, and their softmax weights: exp(l - l_max)/sum in
+ * double, rounded to float. Device pointers: logits float [T*E],
+ * ids int32 [T*k], w float [T*k]. 1 <= k <= 32, k <= E <= 4096.
+ */
+PMOE_API pmoe_status pmoe_route(const float *logits, int T, int E, int k, int32_t *ids, float *w,
+                       pmoe_stream stream);
+
+/*
+ * pmoe_select_prefix [T#29, T#31, A]: per token, depth b_i in 1..8 for each
+ * of its k experts minimising sum w_i^2 * s_e^2 * 4^-b_i under
+ * sum b_i = B = floor(avg_bits*k + 1e-4) clamped to [k, 8k]: all start at 1
+ * bit; B-k times the expert with the largest w_i*s_e*2^-b_i (float product,
+ * exact ldexp compares, ties to the lower slot, 8-bit experts skipped) gets
+ * one more bit. The same as b = clamp(ceil(c + log2(w*s/geomean)), 1, 8)
+ * with the offset c that spends the budget.
+ *   w float [T*k], ids int32 [T*k], sens float [E] (indexed by ids),
+ *   depth uint8 [T*k] out. on_device = 1: device pointers, async on stream;
+ *   0: host pointers, synchronous. 1 <= k <= 32.
+ */
+PMOE_API pmoe_status pmoe_select_prefix(const float *w, const int32_t *ids, const float *sens, int T, int k,
+                               float avg_bits, uint8_t *depth, int on_device, pmoe_stream stream);
+
+/* ------------------------------------------------------------------ */
+/* Execution                                                           */
+/* ------------------------------------------------------------------ */
+
+/* One stored expert matrix (device pointers). */
+typedef struct {
+    const uint32_t *planes;     /* plane p at planes + p*plane_stride_words */
+    int64_t plane_stride_words; /* >= N*K/32 */
+    const float *scales;        /* [N][K/G] */
+    const float *codebook;      /* [510] */
+    int N, K, G;                /* N%16 == 0, K%128 == 0, G in {32, 64, 128} */
+} pmoe_matrix;
+
+/*
+ * pmoe_expert_gemv [T#37, A: Methodology]: y[n] = sum_k scales[n][k/G] *
+ * C[b][code>>(8-b)] * x[k], reading only planes 0..b-1 and decoding in
+ * registers (no dequantised matrix is written).
+ *   x: device, K values, bf16 if x_is_bf16 else float32. y: device float [N].
+ *   1 <= b <= 8. Numerics: weights and x are carried as 16-bit fixed point
+ *   (power-of-two scales per table and per 128 columns), products summed
+ *   exactly in int32 per group, groups in float32.
+ */
+PMOE_API pmoe_status pmoe_expert_gemv(const pmoe_matrix *m, int b, const void *x, int x_is_bf16, float *y,
+                             pmoe_stream stream);
+
+/*
+ * One MoE layer's experts in a plane-slot pool (device pointers).
+ * A slot holds plane p of one expert for all three matrices:
+ *   [gate plane (I x H) | up plane (I x H) | down plane (H x I)], each H*I/32
+ * words, at pool + slot*slot_words. slot_of[e*8 + p] is the slot of plane p
+ * of expert e, or -1 if absent (a depth-b read needs planes 0..b-1 present).
+ * scales: per expert 3 matrices back to back: gate [I][H/G], up [I][H/G],
+ * down [H][I/G]. codebooks: per expert 3 x 510 floats (gate, up, down).
+ */
+typedef struct {
+    int E, H, I, G;           /* H%128 == 0, I%128 == 0, G in {32, 64, 128} */
+    const uint32_t *pool;
+    int64_t slot_words;       /* >= 3*H*I/32 */
+    const int32_t *slot_of;   /* [E*8] */
+    const float *scales;      /* [E][2*I*(H/G) + H*(I/G)] */
+    const float *codebooks;   /* [E][3][510] */
+} pmoe_layer;
+
+/* Workspace needed by pmoe_moe_layer_fwd / pmoe_moe_decode_step for T tokens, top-k. */
+PMOE_API size_t pmoe_layer_workspace_bytes(int T, int k, int E, int H, int I);
+
+/*
+ * pmoe_moe_layer_fwd [T#4, T#37, A]: for each token t and slot i with expert
+ * e = ids[t*k+i] at depth b = depth[t*k+i]:
+ *   g = Wg_b x_t, u = Wu_b x_t, h = silu(g)*u, y_t += w[t*k+i] * (Wd_b h),
+ * with (token, expert) pairs grouped by expert so that tokens at different
+ * depths of one expert share one read of the planes they have in common.
+ *   x: device bf16 [T*H]. ids, w, depth: device [T*k]. y: device float [T*H]
+ *   (overwritten). ws: device scratch of >= pmoe_layer_workspace_bytes().
+ *   Expert ids must be distinct within a token. Output is deterministic (the
+ *   k contributions are summed in slot order).
+ */
+PMOE_API pmoe_status pmoe_moe_layer_fwd(const pmoe_layer *L, const uint16_t *x, const int32_t *ids,
+                               const float *w, const uint8_t *depth, int T, int k, float *y,
+                               void *ws, size_t ws_bytes, pmoe_stream stream);
+
+/*
+ * pmoe_moe_decode_step: the whole hot path for T tokens on the device:
+ * pmoe_route, then pmoe_select_prefix (sens indexed by expert id), then
+ * pmoe_moe_layer_fwd. ids_out, w_out, depth_out: device [T*k], written (may
+ * be NULL to keep them in the workspace only).
+ */
+PMOE_API pmoe_status pmoe_moe_decode_step(const pmoe_layer *L, const float *logits, const float *sens,
+                                 const uint16_t *x, int T, int k, float avg_bits, float *y,
+                                 int32_t *ids_out, float *w_out, uint8_t *depth_out, void *ws,
+                                 size_t ws_bytes, pmoe_stream stream);
+
+/*
+ * pmoe_profile_events: when both events are non-NULL, every later
+ * pmoe_moe_layer_fwd / pmoe_moe_decode_step call on this host thread records
+ * `start` on its stream just before the expert kernels (gate/up + SwiGLU and
+ * down) and `stop` just after them, so cudaEventElapsedTime gives their
+ * device time without routing, grouping and combine. NULL, NULL turns it
+ * off. The events are the caller's (cudaEventCreate); nothing is kept beyond
+ * the two handles.
+ */
+PMOE_API pmoe_status pmoe_profile_events(pmoe_event start, pmoe_event stop);
+
+/*
+ * Materialise-then-multiply ablation [T#37, A: Results]: decodes the depth-b
+ * prefixes of every selected expert to bf16 matrices in the workspace (the
+ * dequantised weights scale*C rounded to bf16), then runs plain GEMVs
+ * (bf16 x bf16, float accumulation) for gate/up, SwiGLU, down and the
+ * weighted combine. Same arguments and output as pmoe_moe_layer_fwd.
+ */
+PMOE_API size_t pmoe_materialise_workspace_bytes(int T, int k, int E, int H, int I);
+PMOE_API pmoe_status pmoe_materialise_layer_fwd(const pmoe_layer *L, const uint16_t *x, const int32_t *ids,
+                                       const float *w, const uint8_t *depth, int T, int k,
+                                       float *y, void *ws, size_t ws_bytes, pmoe_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PMOE_H */

@@ -104,7 +104,8 @@ void or_tree_codebook_f32(float *cb /* [510] */)
  * deviation of the group's weights about their mean, in double, rounded to
  * float; a zero scale becomes 1. code = #{ i in 1..255 : w/scale >= t_i },
  * t_i = Phi^-1(i/256): the index of the equiprobable bin, half-open on the
- * right, so a value exactly on a threshold goes to the upper bin.
+ * right, so a value exactly on a threshold goes to the upper bin. (The count
+ * is taken by bisection over the sorted thresholds.)
  * The reconstruction at depth b is scale * C[b][code >> (8-b)].
  * Pins: hand examples on thresholds; chi-square uniformity of codes on
  * N(0,1) data; scales against numpy's population std.
@@ -141,11 +142,17 @@ void or_quantize(const float *w, int N, int K, int G, float *scales /* [N*(K/G)]
             scales[(size_t)n * ng + g] = s;
             for (int k = 0; k < G; ++k) {
                 double z = (double)src[k] / (double)s;
-                int c = 0;
-                for (int i = 1; i < 256; ++i)
-                    if (z >= t[i])
-                        c = i;
-                codes[(size_t)n * K + (size_t)g * G + k] = (uint8_t)c;
+                /* #{i in 1..255 : t_i <= z}; the thresholds are sorted, so the
+                 * count is found by bisection over them */
+                int lo = 0, hi = 256; /* t[lo] <= z < t[hi] (t[256] = +inf) */
+                while (hi - lo > 1) {
+                    int mid = (lo + hi) / 2;
+                    if (t[mid] <= z)
+                        lo = mid;
+                    else
+                        hi = mid;
+                }
+                codes[(size_t)n * K + (size_t)g * G + k] = (uint8_t)lo;
             }
         }
     }

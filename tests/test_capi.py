@@ -1,0 +1,90 @@
+"""The C-ABI library without a GPU: it loads, exports every declared symbol,
+and its host-side paths agree with the oracle bit for bit."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def pm():
+    from bitplane_mixed_precision_b200 import build
+    build.build()
+    import bitplane_mixed_precision_b200 as pm
+    return pm
+
+
+def declared_symbols():
+    names = []
+    with open(os.path.join(ROOT, "include", "pmoe.h")) as f:
+        text = f.read()
+    for m in re.finditer(r"PMOE_API\s+[\w\s\*]+?\b(pmoe_\w+)\s*\(", text):
+        names.append(m.group(1))
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol(pm):
+    lib = ctypes.CDLL(pm.LIB_PATH)
+    names = declared_symbols()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+    # the binding wraps exactly the declared entry points
+    assert sorted(pm.exported_symbols()) == names
+
+
+def test_codebook_matches_oracle(pm, oracle_mod):
+    cb = np.empty(510, np.float32)
+    pm.tree_codebook(cb)
+    np.testing.assert_array_equal(cb, oracle_mod.tree_codebook_f32())
+
+
+@pytest.mark.parametrize("N,K,depth", [(16, 128, 8), (48, 384, 3), (32, 256, 1), (64, 640, 5)])
+def test_host_pack_matches_oracle(pm, oracle_mod, N, K, depth):
+    rng = np.random.default_rng(N + K + depth)
+    codes = rng.integers(0, 256, size=(N, K), dtype=np.uint8)
+    ref = oracle_mod.pack(codes, depth)
+    stride = N * K // 32 + 64  # planes spaced wider than needed
+    out = np.full(stride * depth, 0xDEADBEEF, dtype=np.uint32)
+    pm.pack_bitplanes(codes, N, K, depth, out, stride, on_device=False)
+    for p in range(depth):
+        np.testing.assert_array_equal(out[p * stride: p * stride + N * K // 32], ref[p])
+        assert np.all(out[p * stride + N * K // 32: (p + 1) * stride] == 0xDEADBEEF)
+
+
+@pytest.mark.parametrize("k,avg", [(10, 2.5), (8, 2.5), (4, 3.25), (16, 1.0), (3, 8.0)])
+def test_host_select_matches_oracle(pm, oracle_mod, synth_mod, k, avg):
+    E, T = 512, 300
+    sens = synth_mod.sensitivities(5, 0, E)
+    logits = np.stack([synth_mod.router_logits(5, t, 0, E) for t in range(T)])
+    ids, w = oracle_mod.route(logits, k)
+    ref = oracle_mod.select(w, ids, sens, avg)
+    out = np.empty((T, k), np.uint8)
+    pm.select_prefix(w, ids, sens, T, k, avg, out, on_device=False)
+    np.testing.assert_array_equal(out, ref)
+
+
+def test_invalid_arguments_are_rejected_on_the_host(pm):
+    codes = np.zeros((15, 128), np.uint8)
+    out = np.zeros(64 * 8, np.uint32)
+    with pytest.raises(pm.PmoeError) as ei:
+        pm.pack_bitplanes(codes, 15, 128, 8, out, 60, on_device=False)
+    assert ei.value.code == 1
+    with pytest.raises(pm.PmoeError):
+        pm.tree_codebook(None)
+    w = np.zeros((1, 40), np.float32)
+    with pytest.raises(pm.PmoeError):
+        pm.select_prefix(w, np.zeros((1, 40), np.int32), np.ones(8, np.float32), 1, 40, 2.5,
+                         np.zeros(40, np.uint8), on_device=False)
+
+
+def test_workspace_queries(pm):
+    a = pm.layer_workspace_bytes(1, 10, 512, 4096, 1024)
+    b = pm.layer_workspace_bytes(32, 10, 512, 4096, 1024)
+    assert 0 < a < b
+    m = pm.materialise_workspace_bytes(1, 10, 512, 4096, 1024)
+    assert m >= 10 * 3 * 4096 * 1024 * 2  # bf16 copies of the ten selected experts

@@ -156,3 +156,13 @@ def test_storage_accounting_golden():
     assert rows["prefix_store"] == (planes_bits, planes_bits // 4)
     indep = sum(range(1, 9))
     assert rows["independent_1_to_8"] == (indep, indep // 4)
+
+
+def test_codes_equal_threshold_count(oracle_mod, synth_mod):
+    """code = #{i in 1..255 : t_i <= w/scale}, checked with numpy's searchsorted."""
+    w = synth_mod.expert_weights(21, 0, 2, 1, 64, 512)
+    scales, codes = oracle_mod.quantize(w, 128)
+    t = oracle_mod.thresholds()[1:]
+    z = w.astype(np.float64) / np.repeat(scales.astype(np.float64), 128, axis=1)
+    ref = np.searchsorted(t, z, side="right")
+    np.testing.assert_array_equal(codes, ref.astype(np.uint8))
