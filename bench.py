@@ -289,6 +289,10 @@ def main():
     ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(N_TOKENS)]
     ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(N_TOKENS)]
     n_prof = min(N_TOKENS, 512)
+    for i in range(n_prof):  # torch creates the underlying cudaEvent at the first record
+        ev0[i].record()
+        ev1[i].record()
+    torch.cuda.synchronize()
     for i in range(n_prof):
         flush.fill_(i & 0xFF)
         pm.profile_events(ev0[i], ev1[i])

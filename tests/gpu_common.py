@@ -47,7 +47,7 @@ class OracleExperts:
             self.cache[e] = oracle.Expert(codes, scales, [self.cb] * 3)
         return self.cache[e]
 
-    def layer(self, E, ids, w, depth, x64, bf16_weights=False):
+    def run(self, E, ids, w, depth, x64, bf16_weights=False):
         need = {int(e): self.get(int(e)) for e in np.unique(ids)}
         return oracle.moe_layer(need, E, self.H, self.I, self.G, ids, w, depth, x64, bf16_weights)
 

@@ -48,7 +48,7 @@ def check_layer(pm, seed, E, H, I, G, k, T, avg=2.5, bias=None, token0=0):
     dep_ref = oracle.select(w_ref, ids_ref, sens, avg)
     np.testing.assert_array_equal(dep, dep_ref)
     x64 = synth.bf16_to_f32(xb).astype(np.float64)
-    ref = O.layer(E, ids_ref, w_ref, dep_ref, x64)
+    ref = O.run(E, ids_ref, w_ref, dep_ref, x64)
     errs = [assert_close(y[t], ref[t], msg=f"token {t}")[0] for t in range(T)]
     return R, O, max(errs), dep
 
@@ -80,9 +80,33 @@ def test_batched_zipf_ragged_blocks(pm):
 
 
 @pytest.mark.parametrize("avg", [1.0, 4.0, 8.0])
-def test_uniform_depths(pm, avg):
+def test_budget_extremes(pm, avg):
+    """avg 1 and 8 force every expert to 1 and 8 bits; avg 4 spends exactly 4 bits per expert."""
     _, _, _, dep = check_layer(pm, 41, 32, 2048, 768, 128, 8, 2, avg=avg)
-    assert np.all(dep == int(avg))
+    assert np.all(dep.sum(axis=1) == int(avg) * 8)
+    if avg in (1.0, 8.0):
+        assert np.all(dep == int(avg))
+
+
+@pytest.mark.parametrize("b", [4, 1, 8])
+def test_uniform_depth_layer(pm, b):
+    """Uniform b-bit requests through pmoe_moe_layer_fwd (the uniform 4-bit run of the large layer)."""
+    seed, E, H, I, G, k, T = 43, 16, 4096, 1024, 128, 10, 2
+    R = ResidentLayer(E, H, I, G, device_fill(seed))
+    O = OracleExperts(seed, H, I, G)
+    logits, xb = tokens(seed, T, E, H)
+    ids, w = oracle.route(logits, k)
+    dep = np.full((T, k), b, np.uint8)
+    y = torch.empty(T * H, dtype=torch.float32, device="cuda")
+    nbytes = pm.layer_workspace_bytes(T, k, E, H, I)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    pm.moe_layer_fwd(R.layer, torch.from_numpy(xb.view(np.int16)).cuda(), torch.from_numpy(ids).cuda(),
+                     torch.from_numpy(w).cuda(), torch.from_numpy(dep).cuda(), T, k, y, ws, nbytes)
+    torch.cuda.synchronize()
+    ref = O.run(E, ids, w, dep, synth.bf16_to_f32(xb).astype(np.float64))
+    got = y.cpu().numpy().reshape(T, H)
+    for t in range(T):
+        assert_close(got[t], ref[t], msg=f"b={b} token {t}")
 
 
 def test_group_size_64(pm):
@@ -128,7 +152,7 @@ def test_materialise_ablation(pm):
                              torch.from_numpy(w).cuda(), torch.from_numpy(dep).cuda(), T, k, y, ws, nbytes)
     torch.cuda.synchronize()
     x64 = synth.bf16_to_f32(xb).astype(np.float64)
-    ref_bf16 = O.layer(E, ids, w, dep, x64, bf16_weights=True)
+    ref_bf16 = O.run(E, ids, w, dep, x64, bf16_weights=True)
     got = y.cpu().numpy().reshape(T, H)
     for t in range(T):
         assert_close(got[t], ref_bf16[t], msg=f"token {t}")
