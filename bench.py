@@ -277,7 +277,7 @@ def main():
         pm.moe_decode_step(R.layer, logits[j], sens, x[j], T, K_TOP, AVG, y[j], ids[j], wts[j], dep[j],
                            ws, ws_bytes, st)
 
-    kernels_per_step = 7  # route+select, group, prep, gate/up, h-prep, down, combine
+    kernels_per_step = 2  # prep (route, select, group, tables, fragments) + persistent expert kernel
 
     # warm-up (eager)
     for i in range(args.warmup):
@@ -397,7 +397,7 @@ def main():
                              "kernel timing with L2 flushed before each token"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
-                         "kernel": "expert kernels (gate/up+SwiGLU, h fragments, down)",
+                         "kernel": "moe_main_kernel (gate/up+SwiGLU, down, combine)",
                          "peak_kind": f"{pk_kind} hbm_gbs"},
             "bitplane_gbs": bitplane_gbs, "bitplane_frac_of_8000": bitplane_gbs / 8000.0,
             "expert_kernels_us": 1e6 * sum(kdur) / len(kdur),

@@ -52,6 +52,7 @@ _SIGS = {
     "pmoe_moe_decode_step": ([ctypes.POINTER(Layer), P, P, P, i32, i32, f32, P, P, P, P, P, sz, P],
                              i32),
     "pmoe_profile_events": ([P, P], i32),
+    "pmoe_layer_error": ([P, ctypes.POINTER(i32), ctypes.POINTER(i32), P], i32),
     "pmoe_materialise_workspace_bytes": ([i32, i32, i32, i32, i32], sz),
     "pmoe_materialise_layer_fwd": ([ctypes.POINTER(Layer), P, P, P, P, i32, i32, P, P, sz, P], i32),
 }
@@ -170,6 +171,14 @@ def profile_events(start, stop) -> None:
             return None
         return e.cuda_event if hasattr(e, "cuda_event") else int(e)
     _check("pmoe_profile_events", _lib.pmoe_profile_events(h(start), h(stop)))
+
+
+def layer_error(ws, stream=None):
+    """(code, detail) of the device-side error record in a layer workspace (synchronises)."""
+    code, detail = i32(0), i32(0)
+    _check("pmoe_layer_error", _lib.pmoe_layer_error(_ptr(ws), ctypes.byref(code), ctypes.byref(detail),
+                                                     _stream(stream)))
+    return code.value, detail.value
 
 
 def materialise_workspace_bytes(T, k, E, H, I) -> int:

@@ -1,4 +1,4 @@
-// Workspace layout of the layer kernels.
+// Workspace layout and limits of the layer kernels.
 #pragma once
 
 #include <cstddef>
@@ -8,18 +8,32 @@
 
 namespace pmoe {
 
-constexpr int kTabWords = 16 + 256; // h[4], l[4], f, pad | shared-memory table of 256 entries
-constexpr int kFlagError = 0, kFlagBlocks = 1, kFlagUnits = 2;
-constexpr int kMaxPairs = 2048;
+constexpr int kTabWords = 16 + 256; // h[4], l[4], f, pad | table of 256 entries for depth >= 5
+constexpr int kMaxPairs = 2048;     // T*k per call
+constexpr int kMaxBlocksPerUnit = 4;
+
+// flags[] words
+constexpr int kFlagError = 0;  // nonzero: error code (see layer.cu)
+constexpr int kFlagBlocks = 1; // column blocks
+constexpr int kFlagUnits = 2;  // expert units
+constexpr int kFlagSched = 3;  // work counter of the persistent kernel
+constexpr int kFlagWhere = 4;  // detail of the first error
 
 // Device pointers into one layer workspace (see carve_layer_ws).
 struct LayerWs {
-    int *flags;      // [64]: error, number of blocks, number of units
-    int *blk_depth;  // per column block: depth
-    int *blk_nmem;   //   members (1..4)
+    int *flags;      // [64]
+    int *blk_depth;  // per column block (<= 4 pairs of one expert and one depth): depth
+    int *blk_nmem;   //   members
     int *blk_pair;   //   [4] pair index t*k + i of each member
     int *blk_expert; //   expert
-    int *unit_expert, *unit_blk0, *unit_nblk, *unit_bmax; // per unit (expert, <= 8 blocks)
+    int *unit_expert, *unit_blk0, *unit_nblk, *unit_bmax; // per unit (one expert, <= 4 blocks)
+    int *cntA;       // per gate/up item (unit, 32 rows of I): consumer warps finished
+    int *cntH;       // per (unit, 128 rows of I): gate/up items finished
+    int *readyB;     // per unit: 128-row tiles of h turned into fragments
+    int *cntB;       // per down item (unit, 128 rows of H): consumer warps finished
+    int *ycnt;       // [T][H/128]: pairs of a token whose down rows are written
+    float *pA;       // [pairs][I/16][8][2][16]: gate/up partial sums per K-part
+    float *pB;       // [pairs][H/16][2][16]: down partial sums per K-part
     uint32_t *tabs;  // [pairs][3][kTabWords]: decode tables per block and matrix
     uint32_t *xfrag; // [T][H/32][8][2]
     int *xexp;       // [T][H/128]

@@ -1,0 +1,661 @@
+// Persistent expert kernel of the MoE layer (included by layer.cu).
+//
+// One CTA per SM: warp NCW is the producer, warps 0..NCW-1 consume.
+//
+// Producer: takes work items from a global counter (gate/up items first, then
+// down items; units deepest first), publishes each item in a small queue and
+// streams the item's bytes into a ring of 16 KB shared-memory slots with 1-D
+// bulk copies completing on mbarriers: one chunk per (matrix, plane) and a
+// "meta" chunk (the scale rows of the item's matrices and the decode tables of
+// its column blocks), ordered [gate planes | meta | up planes] or
+// [meta | down planes] so that no copy of an item ever waits for a slot the
+// same item still holds.
+//
+// Consumers: every consumer warp takes every item and multiplies its share of
+// the item's tiles. Partial sums go to a shared-memory slot of the item (one
+// slot per queue entry); the warp that finishes last (a shared-memory atomic)
+// reduces them in a fixed order, so results are deterministic, writes
+// h = silu(g) * u (gate/up) or the pair's output rows (down), and moves the
+// global counters: the last gate/up item of a 128-row tile of h converts it
+// to MMA fragments and bumps the unit's ready count; the last pair of a
+// token's 128 output rows sums the k pair outputs into y in slot order. Down
+// items wait (bounded) until their unit's h fragments are all ready. Items with
+// several column blocks (batched tokens) keep their partials in global memory.
+namespace mk {
+
+constexpr int NCW = 16;                    // consumer warps
+constexpr int NTHREADS = (NCW + 1) * 32;
+constexpr int NSLOT = 11;                  // ring slots
+constexpr int CHUNK = 16384;               // bytes per ring slot
+constexpr int QDEPTH = 4;                  // item queue (= partial-sum slots)
+constexpr int RED_WORDS = 2 * 16 * 4;      // per warp: [matrix][row][member]
+constexpr int XS_WORDS = (4096 / 32) * 16; // shared copy of the x fragments (T == 1, H <= 4096)
+constexpr int TAB_BYTES = 64;              // decode-table head copied per (block, matrix)
+constexpr uint64_t kDeadlineNs = 200ull * 1000 * 1000;
+
+struct Desc {
+    int kind; // 0 gate/up, 1 down, 2 stop
+    int u;    // unit
+    int strip;
+    int c0;   // first chunk of the item
+};
+
+struct Smem {
+    alignas(128) unsigned char ring[NSLOT][CHUNK];
+    float red[QDEPTH][NCW][RED_WORDS];
+    uint32_t xs[XS_WORDS];
+    uint32_t zeros[4];
+    int xse[32];
+    uint64_t full[NSLOT], empty[NSLOT], qfull[QDEPTH], qempty[QDEPTH];
+    Desc q[QDEPTH];
+    int cnt[QDEPTH];
+};
+
+struct Args {
+    pmoe_layer L;
+    int T, k;
+    const float *wts; // routing weights [T*k]
+    float *y;         // [T*H]
+    LayerWs W;
+};
+
+// bytes of an item's meta chunk: scales of its rows, then table heads
+__host__ __device__ inline int meta_bytes_gateup(int H, int G, int nblk) { return 2 * 32 * (H / G) * 4 + nblk * 2 * TAB_BYTES; }
+__host__ __device__ inline int meta_bytes_down(int I, int G, int nblk) { return 128 * (I / G) * 4 + nblk * TAB_BYTES; }
+
+__device__ __forceinline__ void set_error(const LayerWs &W, int code, int where)
+{
+    if (atomicCAS(&W.flags[kFlagError], 0, code) == 0)
+        W.flags[kFlagWhere] = where;
+}
+
+__device__ __forceinline__ int atom_add_acq_rel(int *p, int v)
+{
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+__device__ __forceinline__ void red_add_release(int *p, int v)
+{
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void load_tab_smem(const unsigned char *src, RegTab &t)
+{
+    const uint4 a = *reinterpret_cast<const uint4 *>(src);
+    const uint4 b = *reinterpret_cast<const uint4 *>(src + 16);
+    t.h[0] = a.x; t.h[1] = a.y; t.h[2] = a.z; t.h[3] = a.w;
+    t.l[0] = b.x; t.l[1] = b.y; t.l[2] = b.z; t.l[3] = b.w;
+    t.f = *reinterpret_cast<const int *>(src + 32);
+}
+
+// 2^-e as a float (e in [-126, 127]).
+__device__ __forceinline__ float pow2neg(int e) { return __int_as_float((127 - e) << 23); }
+
+// The four int32 partial sums of one row (dh0 = sum vh*xh, dh1 = sum vh*xl,
+// dl0 = sum vl*xh, dl1 = sum vl*xl) as one integer in units of 256 (the
+// vl*xl term rounded to that unit, far below the float resolution of the sum).
+__device__ __forceinline__ float combine256(int dh0, int dh1, int dl0, int dl1)
+{
+    return (float)(dh0 * 256 + dh1 + dl0 + ((dl1 + 128) >> 8));
+}
+
+// B fragment sources: 0 = x fragments in shared memory, 1 = x fragments in
+// global memory (written by the prep kernel), 2 = h fragments in global memory
+// (written by other CTAs of this kernel: read through L2).
+template <int FRAG>
+__device__ __forceinline__ uint2 frag_at(const uint32_t *p)
+{
+    if constexpr (FRAG == 2)
+        return __ldcg(reinterpret_cast<const uint2 *>(p));
+    else if constexpr (FRAG == 1)
+        return __ldg(reinterpret_cast<const uint2 *>(p));
+    else
+        return *reinterpret_cast<const uint2 *>(p);
+}
+
+template <int FRAG>
+__device__ __forceinline__ int exp_at(const int *p)
+{
+    if constexpr (FRAG == 2)
+        return __ldcg(p);
+    else if constexpr (FRAG == 1)
+        return __ldg(p);
+    else
+        return *p;
+}
+
+// One column block over this warp's tiles of one matrix.
+//  pp[p]: plane p's chunk + this warp's first tile + lane offset (shared).
+//  tabs: table head in shared memory; big: full table (global) for depth >= 5.
+//  fptr/fstep: this lane's B-fragment words at the first tile and the step per
+//  k-step in words (FRAG 0: always valid, a zero block for absent members).
+//  exps: exponents of this lane's epilogue member (nullptr: no epilogue).
+//  sc0/sc1: scale rows (shared) of rows g, g+8 at the warp's first group.
+template <int B, int GS, int FRAG>
+__device__ __forceinline__ void warp_block(const unsigned char *const (&pp)[8], int ntiles, int Q0,
+                                           const unsigned char *tabs, const uint32_t *big, const uint32_t *fptr,
+                                           int fstep, const int *exps, const float *sc0, const float *sc1,
+                                           float &acc0, float &acc1)
+{
+    constexpr int NG = 4 / GS; // scale groups per 128-column tile
+    RegTab tab;
+    load_tab_smem(tabs, tab);
+    const bool epi = exps != nullptr;
+    for (int j = 0; j < ntiles; ++j) {
+        uint32_t w[8][2];
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            w[p][0] = w[p][1] = 0u;
+            if (p < B) {
+                const uint2 v = *reinterpret_cast<const uint2 *>(pp[p] + j * 256);
+                w[p][0] = v.x;
+                w[p][1] = v.y;
+            }
+        }
+        const float fac = epi ? 256.0f * pow2neg(tab.f + exp_at<FRAG>(exps + Q0 + j)) : 0.0f;
+        int dh[4] = {0, 0, 0, 0}, dl[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            uint32_t ah[4], al[4];
+            dev::decode_kstep<B>(w, s, tab, big, ah, al);
+            uint2 bv = make_uint2(0u, 0u);
+            if (FRAG == 0 || fptr != nullptr)
+                bv = frag_at<FRAG>(fptr + (j * 4 + s) * fstep);
+            dev::mma_s8(dh, ah, bv.x, bv.y);
+            dev::mma_s8(dl, al, bv.x, bv.y);
+            if ((s + 1) % GS == 0) {
+                const int gi = j * NG + s / GS;
+                acc0 = __fmaf_rn(combine256(dh[0], dh[1], dl[0], dl[1]), sc0[gi] * fac, acc0);
+                acc1 = __fmaf_rn(combine256(dh[2], dh[3], dl[2], dl[3]), sc1[gi] * fac, acc1);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dh[i] = dl[i] = 0;
+            }
+        }
+    }
+}
+
+template <int GS, int FRAG>
+__device__ __forceinline__ void warp_block_any(int d, const unsigned char *const (&pp)[8], int ntiles, int Q0,
+                                               const unsigned char *tabs, const uint32_t *big, const uint32_t *fptr,
+                                               int fstep, const int *exps, const float *sc0, const float *sc1,
+                                               float &acc0, float &acc1)
+{
+    switch (d) {
+    case 1: warp_block<1, GS, FRAG>(pp, ntiles, Q0, tabs, big, fptr, fstep, exps, sc0, sc1, acc0, acc1); break;
+    case 2: warp_block<2, GS, FRAG>(pp, ntiles, Q0, tabs, big, fptr, fstep, exps, sc0, sc1, acc0, acc1); break;
+    case 3: warp_block<3, GS, FRAG>(pp, ntiles, Q0, tabs, big, fptr, fstep, exps, sc0, sc1, acc0, acc1); break;
+    case 4: warp_block<4, GS, FRAG>(pp, ntiles, Q0, tabs, big, fptr, fstep, exps, sc0, sc1, acc0, acc1); break;
+    case 5: warp_block<5, GS, FRAG>(pp, ntiles, Q0, tabs, big, fptr, fstep, exps, sc0, sc1, acc0, acc1); break;
+    case 6: warp_block<6, GS, FRAG>(pp, ntiles, Q0, tabs, big, fptr, fstep, exps, sc0, sc1, acc0, acc1); break;
+    case 7: warp_block<7, GS, FRAG>(pp, ntiles, Q0, tabs, big, fptr, fstep, exps, sc0, sc1, acc0, acc1); break;
+    default: warp_block<8, GS, FRAG>(pp, ntiles, Q0, tabs, big, fptr, fstep, exps, sc0, sc1, acc0, acc1); break;
+    }
+}
+
+// h of one pair, one 128-column tile -> B fragments (one warp); h read through L2.
+__device__ void h_to_frags(const LayerWs &W, int I, int pair, int Q)
+{
+    const int lane = threadIdx.x & 31;
+    const float4 f = __ldcg(reinterpret_cast<const float4 *>(W.h + (int64_t)pair * I + 128 * Q + 4 * lane));
+    float v[4] = {f.x, f.y, f.z, f.w};
+    float m = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+    m = dev::warp_max(m);
+    const int sx = dev::fix_exponent(m);
+    uint32_t ph = 0u, pl = 0u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        int hi, lo;
+        dev::split16(__float2int_rn(ldexpf(v[i], sx)), hi, lo);
+        ph |= (uint32_t)(hi & 0xff) << (8 * i);
+        pl |= (uint32_t)(lo & 0xff) << (8 * i);
+    }
+    const int s = lane >> 3, o = lane & 7, t = o & 3, reg = o >> 2;
+    uint32_t *xf = W.hfrag + (int64_t)pair * (I / 32) * 16;
+    __stcg(xf + ((Q * 4 + s) * 8 + t) * 2 + reg, ph);
+    __stcg(xf + ((Q * 4 + s) * 8 + 4 + t) * 2 + reg, pl);
+    if (lane == 0)
+        __stcg(W.hexp + (int64_t)pair * (I / 128) + Q, sx);
+}
+
+// After the h rows of a gate/up item are written: count the item on its
+// 128-row tile of h; the last one converts the tile and bumps the unit's ready count.
+__device__ void gateup_tile_done(const LayerWs &W, int I, int u, int s32, int blk0, int nblk)
+{
+    const int lane = threadIdx.x & 31;
+    __syncwarp();
+    int last = 0;
+    if (lane == 0)
+        last = (atom_add_acq_rel(&W.cntH[u * (I / 128) + s32 / 4], 1) == 3);
+    last = __shfl_sync(0xffffffffu, last, 0);
+    __syncwarp();
+    if (!last)
+        return;
+    for (int bi = 0; bi < nblk; ++bi) {
+        const int blk = blk0 + bi, nmem = __ldg(W.blk_nmem + blk);
+        for (int c = 0; c < nmem; ++c)
+            h_to_frags(W, I, __ldg(W.blk_pair + blk * 4 + c), s32 / 4);
+    }
+    __syncwarp();
+    if (lane == 0)
+        red_add_release(&W.readyB[u], 1);
+}
+
+// After a pair's 128 output rows are written: the last of the token's k pairs
+// sums them into y in slot order.
+__device__ void down_rows_done(const Args &a, int pair, int s128)
+{
+    const LayerWs &W = a.W;
+    const int lane = threadIdx.x & 31, H = a.L.H, k = a.k;
+    const int tok = pair / k;
+    __syncwarp();
+    int last = 0;
+    if (lane == 0)
+        last = (atom_add_acq_rel(&W.ycnt[tok * (H / 128) + s128], 1) == k - 1);
+    last = __shfl_sync(0xffffffffu, last, 0);
+    __syncwarp();
+    if (!last)
+        return;
+    for (int r = lane; r < 128; r += 32) {
+        float s = 0.0f;
+        for (int i = 0; i < k; ++i)
+            s = __fmaf_rn(__ldg(a.wts + tok * k + i), __ldcg(W.part + (int64_t)(tok * k + i) * H + 128 * s128 + r), s);
+        a.y[(int64_t)tok * H + 128 * s128 + r] = s;
+    }
+}
+
+template <int GS>
+__global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
+{
+    extern __shared__ __align__(128) unsigned char smraw[];
+    Smem &S = *reinterpret_cast<Smem *>(smraw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const pmoe_layer &L = a.L;
+    const LayerWs &W = a.W;
+    const int H = L.H, I = L.I, G = L.G, T = a.T, k = a.k;
+    const uint64_t deadline = pipe::globaltimer() + kDeadlineNs;
+
+    if (tid == 0) {
+        for (int s = 0; s < NSLOT; ++s) {
+            pipe::mbar_init(&S.full[s], 1);
+            pipe::mbar_init(&S.empty[s], NCW);
+        }
+        for (int s = 0; s < QDEPTH; ++s) {
+            pipe::mbar_init(&S.qfull[s], 1);
+            pipe::mbar_init(&S.qempty[s], NCW);
+            S.cnt[s] = 0;
+        }
+        pipe::fence_barrier_init();
+    }
+    if (tid < 4)
+        S.zeros[tid] = 0u;
+    __syncthreads();
+    pipe::wait_prerequisites(); // the prep kernel's results are visible from here on
+
+    const int nunits = W.flags[kFlagUnits];
+    const int SA = I / 32;  // gate/up items per unit (32 rows of I each)
+    const int SB = H / 128; // down items per unit (128 rows of H each)
+    const int totalA = nunits * SA, total = totalA + nunits * SB;
+    const int64_t mat_words = (int64_t)H * I / 32;
+    const int64_t escale_len = 2 * (int64_t)I * (H / G) + (int64_t)H * (I / G);
+    const bool stage_x = (T == 1 && H <= 4096);
+    if (stage_x) {
+        for (int i = tid; i < (H / 32) * 16; i += NTHREADS)
+            S.xs[i] = W.xfrag[i];
+        for (int i = tid; i < H / 128; i += NTHREADS)
+            S.xse[i] = W.xexp[i];
+    }
+    __syncthreads();
+
+    if (warp == NCW) {
+        // ------------------------------------------------------------ producer
+        if (lane != 0)
+            return;
+        int c = 0, qi = 0;
+        bool ok = true;
+        auto next_slot = [&](int &s) {
+            s = c % NSLOT;
+            if (c >= NSLOT && !pipe::mbar_wait(&S.empty[s], ((c / NSLOT) + 1) & 1, deadline)) {
+                set_error(W, kErrTimeout, 2);
+                ok = false;
+            }
+        };
+        while (ok) {
+            Desc d;
+            const int u = atomicAdd(&W.flags[kFlagSched], 1);
+            if (u >= total) {
+                d.kind = 2;
+                d.u = d.strip = 0;
+            } else if (u < totalA) {
+                d.kind = 0;
+                d.u = u / SA;
+                d.strip = u % SA;
+            } else {
+                d.kind = 1;
+                d.u = (u - totalA) / SB;
+                d.strip = (u - totalA) % SB;
+            }
+            d.c0 = c;
+            const int qs = qi % QDEPTH;
+            if (qi >= QDEPTH && !pipe::mbar_wait(&S.qempty[qs], ((qi / QDEPTH) + 1) & 1, deadline)) {
+                set_error(W, kErrTimeout, 1);
+                break;
+            }
+            S.q[qs] = d;
+            pipe::mbar_arrive(&S.qfull[qs]);
+            ++qi;
+            if (d.kind == 2)
+                break;
+            const int e = __ldg(W.unit_expert + d.u), bmax = __ldg(W.unit_bmax + d.u);
+            const int blk0 = __ldg(W.unit_blk0 + d.u), nblk = __ldg(W.unit_nblk + d.u);
+            const float *esc = L.scales + (int64_t)e * escale_len;
+            // chunk order: gate/up items [gate planes | meta | up planes], down items [meta | planes];
+            // an item's own meta slot is never the one its later chunks wait for (2*8+1 > NSLOT).
+            auto issue_planes = [&](int m) {
+                for (int p = 0; p < bmax && ok; ++p) {
+                    int s;
+                    next_slot(s);
+                    if (!ok)
+                        break;
+                    const int slot = __ldg(L.slot_of + e * 8 + p);
+                    uint32_t bytes;
+                    int64_t off;
+                    if (d.kind == 0) {
+                        bytes = (uint32_t)(2 * (H / 128) * 256);
+                        off = m * mat_words + (int64_t)d.strip * 2 * (H / 128) * 64;
+                    } else {
+                        bytes = (uint32_t)(8 * (I / 128) * 256);
+                        off = 2 * mat_words + (int64_t)d.strip * 8 * (I / 128) * 64;
+                    }
+                    if (slot >= 0) {
+                        pipe::mbar_arrive_expect_tx(&S.full[s], bytes);
+                        pipe::bulk_g2s(S.ring[s], L.pool + (int64_t)slot * L.slot_words + off, bytes, &S.full[s]);
+                    } else {
+                        // a missing plane: report it and complete the slot without data
+                        set_error(W, kErrNoPlane, e * 8 + p);
+                        pipe::mbar_arrive(&S.full[s]);
+                    }
+                    ++c;
+                }
+            };
+            auto issue_meta = [&]() {
+                int s;
+                next_slot(s);
+                if (!ok)
+                    return;
+                if (d.kind == 0) {
+                    const uint32_t sb = 32 * (H / G) * 4;
+                    pipe::mbar_arrive_expect_tx(&S.full[s], meta_bytes_gateup(H, G, nblk));
+                    for (int m = 0; m < 2; ++m)
+                        pipe::bulk_g2s(S.ring[s] + m * sb,
+                                       esc + (int64_t)m * I * (H / G) + (int64_t)d.strip * 32 * (H / G), sb, &S.full[s]);
+                    for (int bi = 0; bi < nblk; ++bi)
+                        for (int m = 0; m < 2; ++m)
+                            pipe::bulk_g2s(S.ring[s] + 2 * sb + (bi * 2 + m) * TAB_BYTES,
+                                           W.tabs + ((int64_t)(blk0 + bi) * 3 + m) * kTabWords, TAB_BYTES, &S.full[s]);
+                } else {
+                    const uint32_t sb = 128 * (I / G) * 4;
+                    pipe::mbar_arrive_expect_tx(&S.full[s], meta_bytes_down(I, G, nblk));
+                    pipe::bulk_g2s(S.ring[s], esc + 2 * (int64_t)I * (H / G) + (int64_t)d.strip * 128 * (I / G), sb,
+                                   &S.full[s]);
+                    for (int bi = 0; bi < nblk; ++bi)
+                        pipe::bulk_g2s(S.ring[s] + sb + bi * TAB_BYTES,
+                                       W.tabs + ((int64_t)(blk0 + bi) * 3 + 2) * kTabWords, TAB_BYTES, &S.full[s]);
+                }
+                ++c;
+            };
+            if (d.kind == 0) {
+                issue_planes(0);
+                if (ok)
+                    issue_meta();
+                if (ok)
+                    issue_planes(1);
+            } else {
+                issue_meta();
+                if (ok)
+                    issue_planes(0);
+            }
+        }
+        // no copy may still be landing in shared memory when the CTA exits
+        for (int cc = (c > NSLOT ? c - NSLOT : 0); cc < c; ++cc)
+            pipe::mbar_wait(&S.full[cc % NSLOT], (cc / NSLOT) & 1, deadline + kDeadlineNs);
+        return;
+    }
+
+    // ---------------------------------------------------------------- consumers
+    const int g = lane >> 2, t = lane & 3;
+    for (int qi = 0;; ++qi) {
+        const int qs = qi % QDEPTH;
+        if (!pipe::mbar_wait(&S.qfull[qs], (qi / QDEPTH) & 1, deadline)) {
+            set_error(W, kErrTimeout, 3);
+            break;
+        }
+        const Desc d = S.q[qs];
+        if (d.kind == 2)
+            break;
+        const int blk0 = __ldg(W.unit_blk0 + d.u);
+        const int nblk = __ldg(W.unit_nblk + d.u), bmax = __ldg(W.unit_bmax + d.u);
+        const bool fast = (nblk == 1);
+        float *red = S.red[qs][warp];
+        bool fine = true;
+        const int cm = (d.kind == 0) ? d.c0 + bmax : d.c0; // meta chunk
+        const unsigned char *meta = S.ring[cm % NSLOT];
+        if (!pipe::mbar_wait(&S.full[cm % NSLOT], (cm / NSLOT) & 1, deadline))
+            fine = false;
+
+        if (d.kind == 0) {
+            // gate/up: warp -> strip sr (of 2 x 16 rows) and K part kp (of 8)
+            const int sr = warp >> 3, kp = warp & 7, tpw = (H / 128) / 8, Q0 = kp * tpw;
+            const int tix0 = sr * (H / 128) + Q0;
+            const int ngr = H / G;
+            for (int m = 0; m < 2; ++m) {
+                const unsigned char *pp[8];
+#pragma unroll
+                for (int p = 0; p < 8; ++p) {
+                    const int cc = d.c0 + m * (bmax + 1) + p;
+                    pp[p] = S.ring[cc % NSLOT] + tix0 * 256 + lane * 8;
+                    if (p < bmax && !pipe::mbar_wait(&S.full[cc % NSLOT], (cc / NSLOT) & 1, deadline))
+                        fine = false;
+                }
+                const float *sc0 = reinterpret_cast<const float *>(meta) + (m * 32 + 16 * sr + g) * ngr + Q0 * (128 / G);
+                const float *sc1 = sc0 + 8 * ngr;
+                for (int bi = 0; bi < nblk; ++bi) {
+                    const int blk = blk0 + bi;
+                    const int dd = __ldg(W.blk_depth + blk), nmem = __ldg(W.blk_nmem + blk);
+                    const int c = g >> 1;
+                    float acc0 = 0.0f, acc1 = 0.0f;
+                    const int *exps = nullptr;
+                    if (t < nmem) {
+                        const int tok = __ldg(W.blk_pair + blk * 4 + t) / k;
+                        exps = stage_x ? S.xse : W.xexp + (int64_t)tok * (H / 128);
+                    }
+                    const unsigned char *tabs = meta + 2 * 32 * ngr * 4 + (bi * 2 + m) * TAB_BYTES;
+                    const uint32_t *big = W.tabs + ((int64_t)blk * 3 + m) * kTabWords + 16;
+                    if (stage_x) {
+                        const bool has = c < nmem;
+                        const uint32_t *fptr = has ? S.xs + Q0 * 64 + (4 * (g & 1) + t) * 2 : S.zeros;
+                        warp_block_any<GS, 0>(dd, pp, tpw, Q0, tabs, big, fptr, has ? 16 : 0, exps, sc0, sc1, acc0,
+                                              acc1);
+                    } else {
+                        const uint32_t *fptr = nullptr;
+                        if (c < nmem) {
+                            const int tok = __ldg(W.blk_pair + blk * 4 + c) / k;
+                            fptr = W.xfrag + (int64_t)tok * (H / 32) * 16 + Q0 * 64 + (4 * (g & 1) + t) * 2;
+                        }
+                        warp_block_any<GS, 1>(dd, pp, tpw, Q0, tabs, big, fptr, 16, exps, sc0, sc1, acc0, acc1);
+                    }
+                    if (t < nmem) {
+                        if (fast) {
+                            red[(m * 16 + g) * 4 + t] = acc0;
+                            red[(m * 16 + g + 8) * 4 + t] = acc1;
+                        } else {
+                            const int pair = __ldg(W.blk_pair + blk * 4 + t);
+                            float *dst = W.pA + (((int64_t)pair * (I / 16) + 2 * d.strip + sr) * 8 + kp) * 32 + m * 16;
+                            __stcg(dst + g, acc0);
+                            __stcg(dst + g + 8, acc1);
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0)
+                    for (int p = 0; p < bmax; ++p)
+                        pipe::mbar_arrive(&S.empty[(d.c0 + m * (bmax + 1) + p) % NSLOT]);
+            }
+            __syncwarp();
+            if (lane == 0)
+                pipe::mbar_arrive(&S.empty[cm % NSLOT]);
+            int last = 0;
+            if (fast) {
+                if (lane == 0) {
+                    __threadfence_block();
+                    last = (atomicAdd(&S.cnt[qs], 1) == NCW - 1);
+                }
+            } else if (lane == 0) {
+                last = (atom_add_acq_rel(&W.cntA[d.u * SA + d.strip], 1) == NCW - 1);
+            }
+            last = __shfl_sync(0xffffffffu, last, 0);
+            __syncwarp();
+            if (last) {
+                // h rows of the item: lane = row (32 rows), every member of every block
+                if (fast)
+                    __threadfence_block();
+                for (int bi = 0; bi < nblk; ++bi) {
+                    const int blk = blk0 + bi, nmem = __ldg(W.blk_nmem + blk);
+                    for (int c = 0; c < nmem; ++c) {
+                        const int pair = __ldg(W.blk_pair + blk * 4 + c);
+                        const int s16 = lane >> 4, rr = lane & 15;
+                        float gv = 0.0f, uv = 0.0f;
+                        if (fast) {
+#pragma unroll
+                            for (int kq = 0; kq < 8; ++kq) {
+                                gv += S.red[qs][8 * s16 + kq][(0 * 16 + rr) * 4 + c];
+                                uv += S.red[qs][8 * s16 + kq][(1 * 16 + rr) * 4 + c];
+                            }
+                        } else {
+                            const float *src = W.pA + (((int64_t)pair * (I / 16) + 2 * d.strip + s16) * 8) * 32;
+#pragma unroll
+                            for (int kq = 0; kq < 8; ++kq) {
+                                gv += __ldcg(src + kq * 32 + rr);
+                                uv += __ldcg(src + kq * 32 + 16 + rr);
+                            }
+                        }
+                        __stcg(W.h + (int64_t)pair * I + 32 * d.strip + lane, gv / (1.0f + expf(-gv)) * uv);
+                    }
+                }
+                if (fast && lane == 0)
+                    S.cnt[qs] = 0;
+                gateup_tile_done(W, I, d.u, d.strip, blk0, nblk);
+            }
+        } else {
+            // down: warp -> strip sb (of 8 x 16 rows) and K part kp (of 2)
+            const int sb = warp >> 1, kp = warp & 1, tpw = (I / 128) / 2, Q0 = kp * tpw;
+            const int tix0 = sb * (I / 128) + Q0;
+            const int ngr = I / G;
+            if (lane == 0) {
+                while (pipe::ld_acquire(&W.readyB[d.u]) < I / 128) {
+                    if (pipe::globaltimer() > deadline) {
+                        fine = false;
+                        break;
+                    }
+                    __nanosleep(32);
+                }
+            }
+            fine = __shfl_sync(0xffffffffu, (int)fine, 0) != 0;
+            __syncwarp();
+            const unsigned char *pp[8];
+#pragma unroll
+            for (int p = 0; p < 8; ++p) {
+                const int cc = d.c0 + 1 + p;
+                pp[p] = S.ring[cc % NSLOT] + tix0 * 256 + lane * 8;
+                if (p < bmax && !pipe::mbar_wait(&S.full[cc % NSLOT], (cc / NSLOT) & 1, deadline))
+                    fine = false;
+            }
+            const float *sc0 = reinterpret_cast<const float *>(meta) + (16 * sb + g) * ngr + Q0 * (128 / G);
+            const float *sc1 = sc0 + 8 * ngr;
+            for (int bi = 0; bi < nblk; ++bi) {
+                const int blk = blk0 + bi;
+                const int dd = __ldg(W.blk_depth + blk), nmem = __ldg(W.blk_nmem + blk);
+                const int c = g >> 1;
+                const uint32_t *fptr = nullptr;
+                if (c < nmem) {
+                    const int pair = __ldg(W.blk_pair + blk * 4 + c);
+                    fptr = W.hfrag + (int64_t)pair * (I / 32) * 16 + Q0 * 64 + (4 * (g & 1) + t) * 2;
+                }
+                const int *exps = nullptr;
+                if (t < nmem)
+                    exps = W.hexp + (int64_t)__ldg(W.blk_pair + blk * 4 + t) * (I / 128);
+                float acc0 = 0.0f, acc1 = 0.0f;
+                const unsigned char *tabs = meta + 128 * ngr * 4 + bi * TAB_BYTES;
+                const uint32_t *big = W.tabs + ((int64_t)blk * 3 + 2) * kTabWords + 16;
+                warp_block_any<GS, 2>(dd, pp, tpw, Q0, tabs, big, fptr, 16, exps, sc0, sc1, acc0, acc1);
+                if (t < nmem) {
+                    if (fast) {
+                        red[g * 4 + t] = acc0;
+                        red[(g + 8) * 4 + t] = acc1;
+                    } else {
+                        const int pair = __ldg(W.blk_pair + blk * 4 + t);
+                        float *dst = W.pB + (((int64_t)pair * (H / 16) + 8 * d.strip + sb) * 2 + kp) * 16;
+                        __stcg(dst + g, acc0);
+                        __stcg(dst + g + 8, acc1);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) {
+                for (int p = 0; p < bmax; ++p)
+                    pipe::mbar_arrive(&S.empty[(d.c0 + 1 + p) % NSLOT]);
+                pipe::mbar_arrive(&S.empty[cm % NSLOT]);
+            }
+            int last = 0;
+            if (fast) {
+                if (lane == 0) {
+                    __threadfence_block();
+                    last = (atomicAdd(&S.cnt[qs], 1) == NCW - 1);
+                }
+            } else if (lane == 0) {
+                last = (atom_add_acq_rel(&W.cntB[d.u * SB + d.strip], 1) == NCW - 1);
+            }
+            last = __shfl_sync(0xffffffffu, last, 0);
+            __syncwarp();
+            if (last) {
+                if (fast)
+                    __threadfence_block();
+                for (int bi = 0; bi < nblk; ++bi) {
+                    const int blk = blk0 + bi, nmem = __ldg(W.blk_nmem + blk);
+                    for (int c = 0; c < nmem; ++c) {
+                        const int pair = __ldg(W.blk_pair + blk * 4 + c);
+                        for (int r = lane; r < 128; r += 32) {
+                            const int s8 = r >> 4, rr = r & 15;
+                            float v;
+                            if (fast) {
+                                v = S.red[qs][2 * s8][rr * 4 + c] + S.red[qs][2 * s8 + 1][rr * 4 + c];
+                            } else {
+                                const float *src = W.pB + (((int64_t)pair * (H / 16) + 8 * d.strip + s8) * 2) * 16;
+                                v = __ldcg(src + rr) + __ldcg(src + 16 + rr);
+                            }
+                            __stcg(W.part + (int64_t)pair * H + 128 * d.strip + r, v);
+                        }
+                    }
+                }
+                if (fast && lane == 0)
+                    S.cnt[qs] = 0;
+                for (int bi = 0; bi < nblk; ++bi) {
+                    const int blk = blk0 + bi, nmem = __ldg(W.blk_nmem + blk);
+                    for (int c = 0; c < nmem; ++c)
+                        down_rows_done(a, __ldg(W.blk_pair + blk * 4 + c), d.strip);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0)
+            pipe::mbar_arrive(&S.qempty[qs]);
+        if (!fine) {
+            set_error(W, kErrTimeout, 4);
+            break;
+        }
+    }
+}
+
+} // namespace mk

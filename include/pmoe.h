@@ -201,11 +201,23 @@ PMOE_API size_t pmoe_layer_workspace_bytes(int T, int k, int E, int H, int I);
  *   x: device bf16 [T*H]. ids, w, depth: device [T*k]. y: device float [T*H]
  *   (overwritten). ws: device scratch of >= pmoe_layer_workspace_bytes().
  *   Expert ids must be distinct within a token. Output is deterministic (the
- *   k contributions are summed in slot order).
+ *   k contributions are summed in slot order). T*k <= 2048.
+ *   Shapes: H % 1024 == 0, H <= 4096, I % 256 == 0, I <= 1024 (else
+ *   PMOE_ERR_UNSUPPORTED). Errors found on the device (an expert id or depth
+ *   out of range, a plane without a slot, a bounded wait that ran out) do not
+ *   stop the call; they are recorded in the workspace: see pmoe_layer_error.
  */
 PMOE_API pmoe_status pmoe_moe_layer_fwd(const pmoe_layer *L, const uint16_t *x, const int32_t *ids,
                                const float *w, const uint8_t *depth, int T, int k, float *y,
                                void *ws, size_t ws_bytes, pmoe_stream stream);
+
+/*
+ * pmoe_layer_error: reads the device-side error record of the last layer call
+ * that used workspace ws (synchronises the stream). code: 0 none, 1 expert id
+ * or depth out of range, 2 a needed plane has no slot (detail = e*8 + plane),
+ * 3 a bounded wait inside the kernel ran out (detail = where).
+ */
+PMOE_API pmoe_status pmoe_layer_error(const void *ws, int *code, int *detail, pmoe_stream stream);
 
 /*
  * pmoe_moe_decode_step: the whole hot path for T tokens on the device:

@@ -32,6 +32,7 @@ def run_step(pm, R, logits, xb, sens, k, avg):
     ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
     pm.moe_decode_step(R.layer, d_logits, d_sens, d_x, T, k, avg, y, ids, w, dep, ws, nbytes)
     torch.cuda.synchronize()
+    assert pm.layer_error(ws) == (0, 0)
     return (y.cpu().numpy().reshape(T, H), ids.cpu().numpy().reshape(T, k),
             w.cpu().numpy().reshape(T, k), dep.cpu().numpy().reshape(T, k))
 
@@ -103,6 +104,7 @@ def test_uniform_depth_layer(pm, b):
     pm.moe_layer_fwd(R.layer, torch.from_numpy(xb.view(np.int16)).cuda(), torch.from_numpy(ids).cuda(),
                      torch.from_numpy(w).cuda(), torch.from_numpy(dep).cuda(), T, k, y, ws, nbytes)
     torch.cuda.synchronize()
+    assert pm.layer_error(ws) == (0, 0)
     ref = O.run(E, ids, w, dep, synth.bf16_to_f32(xb).astype(np.float64))
     got = y.cpu().numpy().reshape(T, H)
     for t in range(T):
@@ -156,3 +158,38 @@ def test_materialise_ablation(pm):
     got = y.cpu().numpy().reshape(T, H)
     for t in range(T):
         assert_close(got[t], ref_bf16[t], msg=f"token {t}")
+
+
+def test_missing_plane_is_reported_not_hung(pm):
+    """A selected expert whose plane has no slot: the call completes and records error 2."""
+    seed, E, H, I, G, k, T = 61, 8, 1024, 256, 128, 2, 1
+    R = ResidentLayer(E, H, I, G, device_fill(seed))
+    ids = np.array([[3, 5]], np.int32)
+    w = np.array([[0.5, 0.5]], np.float32)
+    dep = np.array([[2, 1]], np.uint8)
+    R.slot_of[3 * 8 + 1] = -1  # plane 1 of expert 3 is absent
+    y = torch.empty(T * H, dtype=torch.float32, device="cuda")
+    nbytes = pm.layer_workspace_bytes(T, k, E, H, I)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    xb = synth.activation_bf16(seed, 0, 0, H)
+    pm.moe_layer_fwd(R.layer, torch.from_numpy(xb.view(np.int16)).cuda(), torch.from_numpy(ids).cuda(),
+                     torch.from_numpy(w).cuda(), torch.from_numpy(dep).cuda(), T, k, y, ws, nbytes)
+    code, detail = pm.layer_error(ws)
+    assert code == 2 and detail == 3 * 8 + 1
+    # a complete layer reports no error
+    R.slot_of[3 * 8 + 1] = 3 * 8 + 1
+    pm.moe_layer_fwd(R.layer, torch.from_numpy(xb.view(np.int16)).cuda(), torch.from_numpy(ids).cuda(),
+                     torch.from_numpy(w).cuda(), torch.from_numpy(dep).cuda(), T, k, y, ws, nbytes)
+    assert pm.layer_error(ws) == (0, 0)
+
+
+def test_unsupported_shapes_are_rejected(pm):
+    R = ResidentLayer(4, 1536, 256, 128, device_fill(1), experts=[])
+    need = pm.layer_workspace_bytes(1, 2, 4, 1536, 256)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    with pytest.raises(pm.PmoeError) as ei:
+        pm.moe_layer_fwd(R.layer, torch.zeros(1536, dtype=torch.int16, device="cuda"),
+                         torch.zeros(2, dtype=torch.int32, device="cuda"), torch.zeros(2, device="cuda"),
+                         torch.ones(2, dtype=torch.uint8, device="cuda"), 1, 2,
+                         torch.empty(1536, device="cuda"), ws, need)
+    assert ei.value.code == 7
