@@ -52,6 +52,8 @@ _SIGS = {
     "pmoe_moe_decode_step": ([ctypes.POINTER(Layer), P, P, P, i32, i32, f32, P, P, P, P, P, sz, P],
                              i32),
     "pmoe_profile_events": ([P, P], i32),
+    "pmoe_noalloc_scratch_bytes": ([], sz),
+    "pmoe_moe_layer_fwd_noalloc": ([ctypes.POINTER(Layer), P, P, P, P, i32, i32, P, P], i32),
     "pmoe_layer_error": ([P, ctypes.POINTER(i32), ctypes.POINTER(i32), P], i32),
     "pmoe_materialise_workspace_bytes": ([i32, i32, i32, i32, i32], sz),
     "pmoe_materialise_layer_fwd": ([ctypes.POINTER(Layer), P, P, P, P, i32, i32, P, P, sz, P], i32),
@@ -155,6 +157,16 @@ def moe_layer_fwd(L: Layer, x, ids, w, depth, T, k, y, ws, ws_bytes, stream=None
     _check("pmoe_moe_layer_fwd", _lib.pmoe_moe_layer_fwd(ctypes.byref(L), _ptr(x), _ptr(ids), _ptr(w),
                                                          _ptr(depth), T, k, _ptr(y), _ptr(ws), ws_bytes,
                                                          _stream(stream)))
+
+
+def noalloc_scratch_bytes() -> int:
+    return _lib.pmoe_noalloc_scratch_bytes()
+
+
+def moe_layer_fwd_noalloc(L: Layer, x, ids, w, depth, T, k, y, stream=None) -> None:
+    """pmoe_moe_layer_fwd with the library's fixed scratch array instead of a workspace."""
+    _check("pmoe_moe_layer_fwd_noalloc", _lib.pmoe_moe_layer_fwd_noalloc(
+        ctypes.byref(L), _ptr(x), _ptr(ids), _ptr(w), _ptr(depth), T, k, _ptr(y), _stream(stream)))
 
 
 def moe_decode_step(L: Layer, logits, sens, x, T, k, avg_bits, y, ids_out, w_out, depth_out, ws,

@@ -281,9 +281,9 @@ pmoe_status check_layer(const pmoe_layer *L, int T, int k)
 
 static int g_num_sms[128] = {};
 
-static pmoe_status launch_layer(const pmoe_layer *L, const float *logits, const float *sens, const uint16_t *x,
-                                int32_t *ids, float *w, uint8_t *depth, int T, int k, int B, float *y, void *ws,
-                                size_t ws_bytes, cudaStream_t st)
+pmoe_status launch_layer(const pmoe_layer *L, const float *logits, const float *sens, const uint16_t *x,
+                         int32_t *ids, float *w, uint8_t *depth, int T, int k, int B, float *y, void *ws,
+                         size_t ws_bytes, cudaStream_t st)
 {
     size_t need = 0;
     carve_layer_ws(nullptr, T, k, L->H, L->I, &need);

@@ -4,6 +4,8 @@
 #include <cstddef>
 #include <cstdint>
 
+#include <cuda_runtime.h>
+
 #include "../../include/pmoe.h"
 
 namespace pmoe {
@@ -48,5 +50,10 @@ struct LayerWs {
 
 LayerWs carve_layer_ws(void *ws, int T, int k, int H, int I, size_t *bytes);
 pmoe_status check_layer(const pmoe_layer *L, int T, int k);
+// Enqueues the prep and persistent kernels of one layer call on stream st.
+// logits == nullptr: ids/w/depth are inputs; otherwise they are written.
+pmoe_status launch_layer(const pmoe_layer *L, const float *logits, const float *sens, const uint16_t *x,
+                         int32_t *ids, float *w, uint8_t *depth, int T, int k, int B, float *y, void *ws,
+                         size_t ws_bytes, cudaStream_t st);
 
 } // namespace pmoe

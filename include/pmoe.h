@@ -212,6 +212,33 @@ PMOE_API pmoe_status pmoe_moe_layer_fwd(const pmoe_layer *L, const uint16_t *x, 
                                void *ws, size_t ws_bytes, pmoe_stream stream);
 
 /*
+ * pmoe_moe_layer_fwd_noalloc: the same layer call as pmoe_moe_layer_fwd for
+ * callers that cannot hand the library a device allocation for scratch, for
+ * example an engine that owns all device memory in a fixed pool and forbids
+ * libraries from allocating, or code whose memory budget is fixed before the
+ * library is called. The PagedMoE pages have no counterpart of this entry
+ * point; it only changes where the scratch lives.
+ *   Scratch: a fixed array of pmoe_noalloc_scratch_bytes() bytes inside the
+ *   library's device image. Every GPU that loads the library holds it until
+ *   the process exits. The call itself allocates nothing (no cudaMalloc, no
+ *   cudaFree, no allocating library routine).
+ *   Limit: T, k, H, I must need at most that many workspace bytes
+ *   (pmoe_layer_workspace_bytes); larger requests return PMOE_ERR_WORKSPACE.
+ *   First call on a device: looks up the array's device address once
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   Sharing: all calls on a device use the same array and it keeps the last
+ *   call's contents; each call resets what must start at zero. Calls that
+ *   overlap on the GPU (other streams, or without ordering between them)
+ *   race on the array and give wrong results. pmoe_layer_error cannot read
+ *   this array; check results instead.
+ * Arguments as pmoe_moe_layer_fwd, without ws and ws_bytes.
+ */
+PMOE_API size_t pmoe_noalloc_scratch_bytes(void);
+PMOE_API pmoe_status pmoe_moe_layer_fwd_noalloc(const pmoe_layer *L, const uint16_t *x, const int32_t *ids,
+                                                const float *w, const uint8_t *depth, int T, int k, float *y,
+                                                pmoe_stream stream);
+
+/*
  * pmoe_layer_error: reads the device-side error record of the last layer call
  * that used workspace ws (synchronises the stream). code: 0 none, 1 expert id
  * or depth out of range, 2 a needed plane has no slot (detail = e*8 + plane),
