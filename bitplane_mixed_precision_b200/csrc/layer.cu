@@ -53,7 +53,7 @@ LayerWs carve_layer_ws(void *ws, int T, int k, int H, int I, size_t *bytes)
     const size_t o_tab = take(P * 3 * kTabWords * 4);
     const size_t o_xf = take((size_t)T * (H / 32) * 16 * 4), o_xe = take((size_t)T * (H / 128) * 4);
     const size_t o_h = take(P * I * 4);
-    const size_t o_hf = take(P * (I / 32) * 16 * 4), o_he = take(P * (I / 128) * 4);
+    const size_t o_hf = take(P * (I / 32) * 16 * 4), o_he = take(P * (size_t)hexp_stride(I) * 4);
     const size_t o_part = take(P * H * 4);
     const size_t o_ids = take(P * 4), o_w = take(P * 4), o_dep = take(P);
     if (bytes)
@@ -116,16 +116,18 @@ constexpr int kPrepThreads = 512;
 __global__ void __launch_bounds__(kPrepThreads) layer_prep_kernel(PrepArgs a)
 {
     pipe::launch_dependents();
-    extern __shared__ int sm[]; // [P] sorted pairs | [P] unit order scratch (x4)
+    extern __shared__ int sm[]; // [P] key | [P] sorted pairs | 4 x [P] unit scratch
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
     const int T = a.T, k = a.k, P = T * k, E = a.L.E, H = a.L.H, I = a.L.I;
     LayerWs W = a.W;
+    int *key = sm;           // expert * 16 + (15 - depth), or -1 for a bad pair
+    int *sorted = sm + P;
     if (tid == 0) {
         W.flags[kFlagError] = 0;
         W.flags[kFlagWhere] = 0;
         W.flags[kFlagSched] = 0;
     }
-    // 1. routing and selection (decode step)
+    // 1. routing and selection (decode step); the pairs' keys go to shared memory
     if (a.logits != nullptr) {
         for (int tok = warp; tok < T; tok += nwarps) {
             int id;
@@ -137,35 +139,39 @@ __global__ void __launch_bounds__(kPrepThreads) layer_prep_kernel(PrepArgs a)
                 a.ids[tok * k + lane] = id;
                 a.w[tok * k + lane] = wt;
                 a.depth[tok * k + lane] = (uint8_t)b;
+                key[tok * k + lane] = id * 16 + (15 - b);
             }
+        }
+    } else {
+        for (int p = tid; p < P; p += blockDim.x) {
+            const int e = a.ids[p], d = a.depth[p];
+            key[p] = (e < 0 || e >= E || d < 1 || d > 8) ? -1 : e * 16 + (15 - d);
         }
     }
     __syncthreads();
     // 2. group: rank of every pair under (expert asc, depth desc, pair asc)
-    volatile const int32_t *ids = a.ids;
-    volatile const uint8_t *dep = a.depth;
-    int *sorted = sm;
     for (int p = tid; p < P; p += blockDim.x) {
-        const int e = ids[p], d = dep[p];
+        const int kp = key[p];
         int rank = 0;
         for (int q = 0; q < P; ++q) {
-            const int eq = ids[q], dq = dep[q];
-            rank += (eq < e || (eq == e && (dq > d || (dq == d && q < p)))) ? 1 : 0;
+            const int kq = key[q];
+            rank += (kq < kp || (kq == kp && q < p)) ? 1 : 0;
         }
         sorted[rank] = p;
     }
     __syncthreads();
-    int *u_e = sm + P, *u_b0 = sm + 2 * P, *u_nb = sm + 3 * P, *u_bm = sm + 4 * P;
+    int *u_e = sm + 2 * P, *u_b0 = sm + 3 * P, *u_nb = sm + 4 * P, *u_bm = sm + 5 * P;
     __shared__ int s_nb, s_nu;
     if (tid == 0) {
         int nb = 0, nu = 0, prev_e = -1, prev_d = -1, nmem = 0, ublk = 0, bad = 0;
         for (int r = 0; r < P; ++r) {
             const int p = sorted[r];
-            const int e = ids[p], d = dep[p];
-            if (e < 0 || e >= E || d < 1 || d > 8) {
+            const int kk = key[p];
+            if (kk < 0) {
                 bad = 1;
                 continue;
             }
+            const int e = kk >> 4, d = 15 - (kk & 15);
             const bool new_e = (e != prev_e);
             if (new_e || d != prev_d || nmem == 4) {
                 if (new_e || ublk == kMaxBlocksPerUnit) {
@@ -274,7 +280,9 @@ pmoe_status check_layer(const pmoe_layer *L, int T, int k)
         return PMOE_ERR_UNSUPPORTED;
     // an item's scale rows and table heads travel in one ring slot
     if (mk::meta_bytes_gateup(L->H, L->G, kMaxBlocksPerUnit) > mk::CHUNK ||
-        mk::meta_bytes_down(L->I, L->G, kMaxBlocksPerUnit) > mk::CHUNK || !aligned(L->scales, 16))
+        mk::meta_bytes_down(L->I, L->G, kMaxBlocksPerUnit) > mk::CHUNK ||
+        mk::meta_bytes_down(L->I, L->G, 1) + mk::meta_bytes_down_frags(L->I, 4) > mk::CHUNK ||
+        !aligned(L->scales, 16))
         return PMOE_ERR_UNSUPPORTED;
     return PMOE_OK;
 }
@@ -298,7 +306,10 @@ pmoe_status launch_layer(const pmoe_layer *L, const float *logits, const float *
         PMOE_TRY(launch_status());
     }
     PrepArgs pa{*L, logits, sens, x, T, k, B, ids, w, depth, frags_here ? 1 : 0, W};
-    layer_prep_kernel<<<1, kPrepThreads, 5 * P * sizeof(int), st>>>(pa);
+    const size_t prep_smem = 6 * (size_t)P * sizeof(int);
+    if (prep_smem > 40 * 1024)
+        PMOE_CUDA(cudaFuncSetAttribute(layer_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_smem));
+    layer_prep_kernel<<<1, kPrepThreads, prep_smem, st>>>(pa);
     PMOE_TRY(launch_status());
 
     int dev = 0;

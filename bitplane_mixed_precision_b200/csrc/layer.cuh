@@ -14,6 +14,9 @@ constexpr int kTabWords = 16 + 256; // h[4], l[4], f, pad | table of 256 entries
 constexpr int kMaxPairs = 2048;     // T*k per call
 constexpr int kMaxBlocksPerUnit = 4;
 
+// Row stride (ints) of the h-fragment exponents: I/128 rounded up to 16 bytes.
+__host__ __device__ inline int hexp_stride(int I) { return ((I / 128) + 3) & ~3; }
+
 // flags[] words
 constexpr int kFlagError = 0;  // nonzero: error code (see layer.cu)
 constexpr int kFlagBlocks = 1; // column blocks
@@ -41,7 +44,7 @@ struct LayerWs {
     int *xexp;       // [T][H/128]
     float *h;        // [pairs][I]
     uint32_t *hfrag; // [pairs][I/32][8][2]
-    int *hexp;       // [pairs][I/128]
+    int *hexp;       // [pairs][hexp_stride(I)]
     float *part;     // [pairs][H]: down-projection output of each pair
     int32_t *ids;    // [pairs]: routing results kept by the decode step
     float *w;

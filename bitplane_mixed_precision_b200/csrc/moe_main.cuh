@@ -62,6 +62,8 @@ struct Args {
 // bytes of an item's meta chunk: scales of its rows, then table heads
 __host__ __device__ inline int meta_bytes_gateup(int H, int G, int nblk) { return 2 * 32 * (H / G) * 4 + nblk * 2 * TAB_BYTES; }
 __host__ __device__ inline int meta_bytes_down(int I, int G, int nblk) { return 128 * (I / G) * 4 + nblk * TAB_BYTES; }
+// down items with one column block also carry the members' h fragments and exponents
+__host__ __device__ inline int meta_bytes_down_frags(int I, int nmem) { return nmem * (2 * I + hexp_stride(I) * 4); }
 
 __device__ __forceinline__ void set_error(const LayerWs &W, int code, int where)
 {
@@ -217,7 +219,7 @@ __device__ void h_to_frags(const LayerWs &W, int I, int pair, int Q)
     __stcg(xf + ((Q * 4 + s) * 8 + t) * 2 + reg, ph);
     __stcg(xf + ((Q * 4 + s) * 8 + 4 + t) * 2 + reg, pl);
     if (lane == 0)
-        __stcg(W.hexp + (int64_t)pair * (I / 128) + Q, sx);
+        __stcg(W.hexp + (int64_t)pair * hexp_stride(I) + Q, sx);
 }
 
 // After the h rows of a gate/up item are written: count the item on its
@@ -351,7 +353,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
             const int e = __ldg(W.unit_expert + d.u), bmax = __ldg(W.unit_bmax + d.u);
             const int blk0 = __ldg(W.unit_blk0 + d.u), nblk = __ldg(W.unit_nblk + d.u);
             const float *esc = L.scales + (int64_t)e * escale_len;
-            // chunk order: gate/up items [gate planes | meta | up planes], down items [meta | planes];
+            // chunk order: gate/up items [gate planes | meta | up planes], down items [planes | meta];
             // an item's own meta slot is never the one its later chunks wait for (2*8+1 > NSLOT).
             auto issue_planes = [&](int m) {
                 for (int p = 0; p < bmax && ok; ++p) {
@@ -397,12 +399,32 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                                            W.tabs + ((int64_t)(blk0 + bi) * 3 + m) * kTabWords, TAB_BYTES, &S.full[s]);
                 } else {
                     const uint32_t sb = 128 * (I / G) * 4;
-                    pipe::mbar_arrive_expect_tx(&S.full[s], meta_bytes_down(I, G, nblk));
+                    int nmem = 0;
+                    if (nblk == 1) {
+                        // the h fragments come along: wait (bounded) until the unit's h is converted
+                        nmem = __ldg(W.blk_nmem + blk0);
+                        while (pipe::ld_acquire(&W.readyB[d.u]) < I / 128) {
+                            if (pipe::globaltimer() > deadline) {
+                                set_error(W, kErrTimeout, 5);
+                                break;
+                            }
+                            __nanosleep(32);
+                        }
+                        pipe::fence_proxy_async();
+                    }
+                    pipe::mbar_arrive_expect_tx(&S.full[s], meta_bytes_down(I, G, nblk) + meta_bytes_down_frags(I, nmem));
                     pipe::bulk_g2s(S.ring[s], esc + 2 * (int64_t)I * (H / G) + (int64_t)d.strip * 128 * (I / G), sb,
                                    &S.full[s]);
                     for (int bi = 0; bi < nblk; ++bi)
                         pipe::bulk_g2s(S.ring[s] + sb + bi * TAB_BYTES,
                                        W.tabs + ((int64_t)(blk0 + bi) * 3 + 2) * kTabWords, TAB_BYTES, &S.full[s]);
+                    unsigned char *fb = S.ring[s] + sb + nblk * TAB_BYTES;
+                    for (int c2 = 0; c2 < nmem; ++c2) {
+                        const int pair = __ldg(W.blk_pair + blk0 * 4 + c2);
+                        pipe::bulk_g2s(fb + c2 * 2 * I, W.hfrag + (int64_t)pair * (I / 32) * 16, 2 * I, &S.full[s]);
+                        pipe::bulk_g2s(fb + nmem * 2 * I + c2 * hexp_stride(I) * 4,
+                                       W.hexp + (int64_t)pair * hexp_stride(I), hexp_stride(I) * 4, &S.full[s]);
+                    }
                 }
                 ++c;
             };
@@ -413,9 +435,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                 if (ok)
                     issue_planes(1);
             } else {
-                issue_meta();
+                issue_planes(0);
                 if (ok)
-                    issue_planes(0);
+                    issue_meta();
             }
         }
         // no copy may still be landing in shared memory when the CTA exits
@@ -440,7 +462,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
         const bool fast = (nblk == 1);
         float *red = S.red[qs][warp];
         bool fine = true;
-        const int cm = (d.kind == 0) ? d.c0 + bmax : d.c0; // meta chunk
+        const int cm = d.c0 + bmax; // meta chunk (after the first matrix's planes)
         const unsigned char *meta = S.ring[cm % NSLOT];
         if (!pipe::mbar_wait(&S.full[cm % NSLOT], (cm / NSLOT) & 1, deadline))
             fine = false;
@@ -553,7 +575,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
             const int sb = warp >> 1, kp = warp & 1, tpw = (I / 128) / 2, Q0 = kp * tpw;
             const int tix0 = sb * (I / 128) + Q0;
             const int ngr = I / G;
-            if (lane == 0) {
+            if (!fast && lane == 0) {
                 while (pipe::ld_acquire(&W.readyB[d.u]) < I / 128) {
                     if (pipe::globaltimer() > deadline) {
                         fine = false;
@@ -567,7 +589,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
             const unsigned char *pp[8];
 #pragma unroll
             for (int p = 0; p < 8; ++p) {
-                const int cc = d.c0 + 1 + p;
+                const int cc = d.c0 + p;
                 pp[p] = S.ring[cc % NSLOT] + tix0 * 256 + lane * 8;
                 if (p < bmax && !pipe::mbar_wait(&S.full[cc % NSLOT], (cc / NSLOT) & 1, deadline))
                     fine = false;
@@ -578,18 +600,29 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                 const int blk = blk0 + bi;
                 const int dd = __ldg(W.blk_depth + blk), nmem = __ldg(W.blk_nmem + blk);
                 const int c = g >> 1;
-                const uint32_t *fptr = nullptr;
-                if (c < nmem) {
-                    const int pair = __ldg(W.blk_pair + blk * 4 + c);
-                    fptr = W.hfrag + (int64_t)pair * (I / 32) * 16 + Q0 * 64 + (4 * (g & 1) + t) * 2;
-                }
-                const int *exps = nullptr;
-                if (t < nmem)
-                    exps = W.hexp + (int64_t)__ldg(W.blk_pair + blk * 4 + t) * (I / 128);
                 float acc0 = 0.0f, acc1 = 0.0f;
                 const unsigned char *tabs = meta + 128 * ngr * 4 + bi * TAB_BYTES;
                 const uint32_t *big = W.tabs + ((int64_t)blk * 3 + 2) * kTabWords + 16;
-                warp_block_any<GS, 2>(dd, pp, tpw, Q0, tabs, big, fptr, 16, exps, sc0, sc1, acc0, acc1);
+                if (fast) {
+                    // h fragments and exponents of the members arrived with the meta chunk
+                    const uint32_t *hf = reinterpret_cast<const uint32_t *>(meta + 128 * ngr * 4 + TAB_BYTES);
+                    const int *he = reinterpret_cast<const int *>(hf + nmem * (I / 2));
+                    const bool has = c < nmem;
+                    const uint32_t *fptr = has ? hf + c * (I / 2) + Q0 * 64 + (4 * (g & 1) + t) * 2 : S.zeros;
+                    const int *exps = (t < nmem) ? he + t * hexp_stride(I) : nullptr;
+                    warp_block_any<GS, 0>(dd, pp, tpw, Q0, tabs, big, fptr, has ? 16 : 0, exps, sc0, sc1, acc0,
+                                          acc1);
+                } else {
+                    const uint32_t *fptr = nullptr;
+                    if (c < nmem) {
+                        const int pair = __ldg(W.blk_pair + blk * 4 + c);
+                        fptr = W.hfrag + (int64_t)pair * (I / 32) * 16 + Q0 * 64 + (4 * (g & 1) + t) * 2;
+                    }
+                    const int *exps = nullptr;
+                    if (t < nmem)
+                        exps = W.hexp + (int64_t)__ldg(W.blk_pair + blk * 4 + t) * hexp_stride(I);
+                    warp_block_any<GS, 2>(dd, pp, tpw, Q0, tabs, big, fptr, 16, exps, sc0, sc1, acc0, acc1);
+                }
                 if (t < nmem) {
                     if (fast) {
                         red[g * 4 + t] = acc0;
@@ -605,7 +638,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
             __syncwarp();
             if (lane == 0) {
                 for (int p = 0; p < bmax; ++p)
-                    pipe::mbar_arrive(&S.empty[(d.c0 + 1 + p) % NSLOT]);
+                    pipe::mbar_arrive(&S.empty[(d.c0 + p) % NSLOT]);
                 pipe::mbar_arrive(&S.empty[cm % NSLOT]);
             }
             int last = 0;
