@@ -29,7 +29,6 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer decode tokens/s; achieved HBM GB/s on bitplane bytes vs B200 peak"
-WORKLOAD = "moe_layer_e512_top10_h4096_i1024_g128_avg2.5_batch1"
 E, K_TOP, H, I, G, AVG = 512, 10, 4096, 1024, 128, 2.5
 SEED = 2026
 N_TOKENS = 1024
@@ -45,7 +44,14 @@ def parse():
     ap.add_argument("--impl", default="pmoe", choices=["pmoe", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=400)
+    # a smaller layer of the same shape (fewer experts) and fewer distinct tokens, for profiler captures
+    ap.add_argument("--experts", type=int, default=E)
+    ap.add_argument("--tokens", type=int, default=1024)
     return ap.parse_args()
+
+
+def workload(e):
+    return f"moe_layer_e{e}_top10_h4096_i1024_g128_avg2.5_batch1"
 
 
 def peaks():
@@ -215,7 +221,7 @@ def reference_arm(args):
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / max(args.steps, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": WORKLOAD},
+            "data": "synthetic", "config": {"workload": workload(E)},
             "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                              "sample": f"per step: {rows} rows of one selected expert matrix at its "
                                        f"selected depth (dequantise-then-matvec in double); tokens "
@@ -228,7 +234,9 @@ def reference_arm(args):
 # ----------------------------------------------------------------------------- GPU arm
 
 def main():
+    global E, N_TOKENS
     args = parse()
+    E, N_TOKENS = args.experts, args.tokens
     if args.impl == "reference":
         return reference_arm(args)
 
@@ -390,10 +398,10 @@ def main():
             "warmup": args.warmup, "ms_per_step": elapsed * 1e3 / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "s8 mma / s32 acc / f32",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD, "experts": E, "top_k": K_TOP, "hidden": H, "inter": I,
+            "config": {"workload": workload(E), "experts": E, "top_k": K_TOP, "hidden": H, "inter": I,
                        "group": G, "avg_bits": AVG, "batch": 1, "tokens_distinct": N_TOKENS,
                        "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2 (6.4 GB of resident planes), fresh token per step; "
+                       "l2": f"inputs larger than L2 ({E * 3 * 8 * PLANE_BYTES / 1e9:.1f} GB of resident planes), fresh token per step; "
                              "kernel timing with L2 flushed before each token"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,

@@ -108,6 +108,7 @@ struct PrepArgs {
     float *w;
     uint8_t *depth;
     int frags_here; // 1: this kernel converts x; 0: a separate grid kernel did
+    int n_rw;       // routing warps (decode step), each with E floats of staging
     LayerWs W;
 };
 
@@ -116,7 +117,7 @@ constexpr int kPrepThreads = 512;
 __global__ void __launch_bounds__(kPrepThreads) layer_prep_kernel(PrepArgs a)
 {
     pipe::launch_dependents();
-    extern __shared__ int sm[]; // [P] key | [P] sorted pairs | 4 x [P] unit scratch
+    extern __shared__ int sm[]; // [P] key | [P] sorted pairs | 4 x [P] unit scratch | n_rw x [E] logits
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
     const int T = a.T, k = a.k, P = T * k, E = a.L.E, H = a.L.H, I = a.L.I;
     LayerWs W = a.W;
@@ -127,12 +128,21 @@ __global__ void __launch_bounds__(kPrepThreads) layer_prep_kernel(PrepArgs a)
         W.flags[kFlagWhere] = 0;
         W.flags[kFlagSched] = 0;
     }
-    // 1. routing and selection (decode step); the pairs' keys go to shared memory
-    if (a.logits != nullptr) {
-        for (int tok = warp; tok < T; tok += nwarps) {
+    // 1. routing and selection (decode step) on warps [0, n_rw), the pairs' keys
+    //    to shared memory; meanwhile the other warps convert x and zero counters.
+    const int n_rw = (a.logits != nullptr) ? a.n_rw : 0;
+    if (a.logits == nullptr) {
+        for (int p = tid; p < P; p += blockDim.x) {
+            const int e = a.ids[p], d = a.depth[p];
+            key[p] = (e < 0 || e >= E || d < 1 || d > 8) ? -1 : e * 16 + (15 - d);
+        }
+    }
+    if (warp < n_rw) {
+        float *stage = reinterpret_cast<float *>(sm + 6 * P) + (int64_t)warp * E;
+        for (int tok = warp; tok < T; tok += n_rw) {
             int id;
             float wt;
-            dev::route_token(a.logits + (int64_t)tok * E, E, k, id, wt);
+            dev::route_token(a.logits + (int64_t)tok * E, E, k, stage, id, wt);
             const float v = (lane < k) ? __fmul_rn(wt, __ldg(a.sens + id)) : 0.0f;
             const int b = dev::select_token(v, k, a.B, nullptr);
             if (lane < k) {
@@ -143,10 +153,25 @@ __global__ void __launch_bounds__(kPrepThreads) layer_prep_kernel(PrepArgs a)
             }
         }
     } else {
-        for (int p = tid; p < P; p += blockDim.x) {
-            const int e = a.ids[p], d = a.depth[p];
-            key[p] = (e < 0 || e >= E || d < 1 || d > 8) ? -1 : e * 16 + (15 - d);
+        const int wi = warp - n_rw, nw = nwarps - n_rw;
+        if (a.frags_here) {
+            for (int j = wi; j < T * (H / 128); j += nw) {
+                const int t = j / (H / 128), Q = j % (H / 128);
+                dev::make_xfrag_tile<true>(a.x + (int64_t)t * H, Q, W.xfrag + (int64_t)t * (H / 32) * 16,
+                                           W.xexp + (int64_t)t * (H / 128));
+            }
         }
+        const int ti = tid - 32 * n_rw, nt = 32 * nw;
+        for (int i = ti; i < P * (I / 32); i += nt)
+            W.cntA[i] = 0;
+        for (int i = ti; i < P * (I / 128); i += nt)
+            W.cntH[i] = 0;
+        for (int i = ti; i < P * (H / 128); i += nt)
+            W.cntB[i] = 0;
+        for (int i = ti; i < P; i += nt)
+            W.readyB[i] = 0;
+        for (int i = ti; i < T * (H / 128); i += nt)
+            W.ycnt[i] = 0;
     }
     __syncthreads();
     // 2. group: rank of every pair under (expert asc, depth desc, pair asc)
@@ -212,16 +237,7 @@ __global__ void __launch_bounds__(kPrepThreads) layer_prep_kernel(PrepArgs a)
         W.unit_blk0[rank] = u_b0[i];
         W.unit_nblk[rank] = u_nb[i];
         W.unit_bmax[rank] = u_bm[i];
-        W.readyB[rank] = 0;
     }
-    for (int i = tid; i < nu * (I / 32); i += blockDim.x)
-        W.cntA[i] = 0;
-    for (int i = tid; i < nu * (I / 128); i += blockDim.x)
-        W.cntH[i] = 0;
-    for (int i = tid; i < nu * (H / 128); i += blockDim.x)
-        W.cntB[i] = 0;
-    for (int i = tid; i < T * (H / 128); i += blockDim.x)
-        W.ycnt[i] = 0;
     // 4. decode tables: one warp per (block, matrix)
     for (int j = warp; j < nb * 3; j += nwarps) {
         const int blk = j / 3, m = j % 3;
@@ -230,19 +246,12 @@ __global__ void __launch_bounds__(kPrepThreads) layer_prep_kernel(PrepArgs a)
         RegTab tab;
         dev::build_tab(a.L.codebooks + ((int64_t)e * 3 + m) * 510, d, tab, d >= 5 ? dst + 16 : nullptr);
         if (lane < 4) {
-            dst[lane] = tab.h[lane];
-            dst[4 + lane] = tab.l[lane];
+            const int r = lane;
+            dst[r] = r == 0 ? tab.h[0] : r == 1 ? tab.h[1] : r == 2 ? tab.h[2] : tab.h[3];
+            dst[4 + r] = r == 0 ? tab.l[0] : r == 1 ? tab.l[1] : r == 2 ? tab.l[2] : tab.l[3];
         }
         if (lane == 0)
             dst[8] = (uint32_t)tab.f;
-    }
-    // 5. activation fragments
-    if (a.frags_here) {
-        for (int j = warp; j < T * (H / 128); j += nwarps) {
-            const int t = j / (H / 128), Q = j % (H / 128);
-            dev::make_xfrag_tile<true>(a.x + (int64_t)t * H, Q, W.xfrag + (int64_t)t * (H / 32) * 16,
-                                       W.xexp + (int64_t)t * (H / 128));
-        }
     }
 }
 
@@ -305,8 +314,17 @@ pmoe_status launch_layer(const pmoe_layer *L, const float *logits, const float *
         xfrag_kernel<<<(warps + 7) / 8, 256, 0, st>>>(x, T, L->H, W);
         PMOE_TRY(launch_status());
     }
-    PrepArgs pa{*L, logits, sens, x, T, k, B, ids, w, depth, frags_here ? 1 : 0, W};
-    const size_t prep_smem = 6 * (size_t)P * sizeof(int);
+    // routing warps: at most one per token, one warp left for the x fragments, E floats each
+    int n_rw = 0;
+    if (logits != nullptr) {
+        n_rw = (kPrepThreads / 32) - 1;
+        n_rw = n_rw < T ? n_rw : T;
+        const int cap = (int)((32 * 1024) / ((size_t)L->E * sizeof(float)));
+        n_rw = n_rw < cap ? n_rw : cap;
+        n_rw = n_rw > 1 ? n_rw : 1;
+    }
+    PrepArgs pa{*L, logits, sens, x, T, k, B, ids, w, depth, frags_here ? 1 : 0, n_rw, W};
+    const size_t prep_smem = 6 * (size_t)P * sizeof(int) + (size_t)n_rw * L->E * sizeof(float);
     if (prep_smem > 40 * 1024)
         PMOE_CUDA(cudaFuncSetAttribute(layer_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_smem));
     layer_prep_kernel<<<1, kPrepThreads, prep_smem, st>>>(pa);

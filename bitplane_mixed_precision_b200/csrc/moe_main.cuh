@@ -25,9 +25,9 @@ namespace mk {
 
 constexpr int NCW = 16;                    // consumer warps
 constexpr int NTHREADS = (NCW + 1) * 32;
-constexpr int NSLOT = 11;                  // ring slots
+constexpr int NSLOT = 12;                  // ring slots
 constexpr int CHUNK = 16384;               // bytes per ring slot
-constexpr int QDEPTH = 4;                  // item queue (= partial-sum slots)
+constexpr int QDEPTH = 2;                  // item queue (= partial-sum slots): claim at most one item ahead
 constexpr int RED_WORDS = 2 * 16 * 4;      // per warp: [matrix][row][member]
 constexpr int XS_WORDS = (4096 / 32) * 16; // shared copy of the x fragments (T == 1, H <= 4096)
 constexpr int TAB_BYTES = 64;              // decode-table head copied per (block, matrix)
@@ -50,6 +50,7 @@ struct Smem {
     Desc q[QDEPTH];
     int cnt[QDEPTH];
 };
+static_assert(sizeof(Smem) <= 227 * 1024, "shared memory of the persistent kernel exceeds one SM's");
 
 struct Args {
     pmoe_layer L;
@@ -354,7 +355,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
             const int blk0 = __ldg(W.unit_blk0 + d.u), nblk = __ldg(W.unit_nblk + d.u);
             const float *esc = L.scales + (int64_t)e * escale_len;
             // chunk order: gate/up items [gate planes | meta | up planes], down items [planes | meta];
-            // an item's own meta slot is never the one its later chunks wait for (2*8+1 > NSLOT).
+            // an item's own meta slot is never the one its later chunks wait for (8 < NSLOT).
             auto issue_planes = [&](int m) {
                 for (int p = 0; p < bmax && ok; ++p) {
                     int s;

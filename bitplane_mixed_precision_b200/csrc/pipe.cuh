@@ -60,13 +60,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 // deadline (global timer, ns) passed first.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t deadline)
 {
-    if (mbar_try_wait(bar, parity))
-        return true;
-    while (!mbar_try_wait(bar, parity)) {
-        if (globaltimer() > deadline)
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if ((n & 15u) == 0 && globaltimer() > deadline)
             return false;
     }
-    return true;
 }
 
 // Bulk copy global -> shared (this CTA), completion counted on bar in bytes.

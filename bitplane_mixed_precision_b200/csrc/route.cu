@@ -44,16 +44,18 @@ static void select_host(const float *w, const int32_t *ids, const float *sens, i
 
 // ---------------------------------------------------------------- device kernels
 
-// One warp per token; see route.cuh for the two device functions.
+// One warp (block) per token, its logits staged in shared memory; see
+// route.cuh for the device functions.
 __global__ void route_kernel(const float *__restrict__ logits, int T, int E, int k,
                              int32_t *__restrict__ ids, float *__restrict__ w)
 {
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    extern __shared__ float stage[];
+    const int warp = blockIdx.x;
     if (warp >= T)
         return;
     int id;
     float wt;
-    dev::route_token(logits + (int64_t)warp * E, E, k, id, wt);
+    dev::route_token(logits + (int64_t)warp * E, E, k, stage, id, wt);
     const int lane = threadIdx.x & 31;
     if (lane < k) {
         ids[warp * k + lane] = id;
@@ -91,8 +93,7 @@ pmoe_status pmoe_route(const float *logits, int T, int E, int k, int32_t *ids, f
         return PMOE_ERR_INVALID_ARG;
     if (T == 0)
         return PMOE_OK;
-    const int blocks = (T + 3) / 4;
-    route_kernel<<<blocks, 128, 0, (cudaStream_t)stream>>>(logits, T, E, k, ids, w);
+    route_kernel<<<T, 32, (size_t)E * sizeof(float), (cudaStream_t)stream>>>(logits, T, E, k, ids, w);
     return launch_status();
 }
 

@@ -18,18 +18,21 @@ __device__ __forceinline__ uint32_t ord_key(float f)
 // Top-k of l[0..E) (ties to the lower id), descending, and softmax over the k
 // (PagedMoE transcript cue 4: k experts, weights summing to one). Executed by
 // a full warp; lane s < k receives slot s. Lane c holds ids c, c+32, ...
-__device__ __forceinline__ void route_token(const float *__restrict__ l, int E, int k, int &id_out,
+// stage: E floats of shared memory for this warp; the logits are copied there
+// once so that the rescans after each pick read shared memory.
+__device__ __forceinline__ void route_token(const float *__restrict__ l, int E, int k, float *stage, int &id_out,
                                             float &w_out)
 {
     const int lane = threadIdx.x & 31;
-    uint32_t taken[4] = {0u, 0u, 0u, 0u}; // E <= 4096: 128 ids per lane
+    for (int j = lane; j < E; j += 32)
+        stage[j] = __ldg(l + j);
+    __syncwarp();
+    // a picked id is overwritten with the bit pattern whose key is 0 (never picked)
     auto local_best = [&](uint32_t &bk, int &bj) {
         bk = 0u;
         bj = -1;
         for (int j = 0; lane + 32 * j < E; ++j) {
-            if ((taken[j >> 5] >> (j & 31)) & 1u)
-                continue;
-            const uint32_t key = ord_key(__ldg(l + lane + 32 * j));
+            const uint32_t key = ord_key(stage[lane + 32 * j]);
             if (key > bk) {
                 bk = key;
                 bj = j;
@@ -40,21 +43,19 @@ __device__ __forceinline__ void route_token(const float *__restrict__ l, int E, 
     int bj;
     local_best(bk, bj);
     int my_id = 0;
-    float my_l = 0.0f;
     for (int s = 0; s < k; ++s) {
         const uint32_t gmax = __reduce_max_sync(0xffffffffu, bk);
         const unsigned cand = (bj >= 0 && bk == gmax) ? (unsigned)(lane + 32 * bj) : 0x7fffffffu;
         const unsigned win = __reduce_min_sync(0xffffffffu, cand);
-        if (lane == s) {
+        if (lane == s)
             my_id = (int)win;
-            my_l = __ldg(l + win);
-        }
         if (lane == (int)(win & 31u)) {
-            const int j = (int)(win >> 5);
-            taken[j >> 5] |= 1u << (j & 31);
+            stage[win] = __uint_as_float(0xffffffffu);
             local_best(bk, bj);
         }
     }
+    const float my_l = (lane < k) ? __ldg(l + my_id) : 0.0f;
+    __syncwarp();
     const double l0 = (double)__shfl_sync(0xffffffffu, my_l, 0);
     const double e = (lane < k) ? exp((double)my_l - l0) : 0.0;
     double sum = 0.0;
