@@ -36,6 +36,15 @@ class Layer(ctypes.Structure):
                 ("slot_of", P), ("scales", P), ("codebooks", P)]
 
 
+class CacheStats(ctypes.Structure):
+    """pmoe_cache_stats: accumulated prefix-cache counters."""
+    _fields_ = [("requests", i64), ("hits", i64), ("planes_fetched", i64), ("bytes_fetched", i64),
+                ("planes_evicted", i64)]
+
+    def as_dict(self):
+        return {n: getattr(self, n) for n, _ in self._fields_}
+
+
 _SIGS = {
     "pmoe_status_string": ([i32], ctypes.c_char_p),
     "pmoe_last_cuda_error": ([], i32),
@@ -57,6 +66,15 @@ _SIGS = {
     "pmoe_layer_error": ([P, ctypes.POINTER(i32), ctypes.POINTER(i32), P], i32),
     "pmoe_materialise_workspace_bytes": ([i32, i32, i32, i32, i32], sz),
     "pmoe_materialise_layer_fwd": ([ctypes.POINTER(Layer), P, P, P, P, i32, i32, P, P, sz, P], i32),
+    "pmoe_cache_create": ([i32, i32, i64, i64, P, P, i32, ctypes.POINTER(P)], i32),
+    "pmoe_cache_extend": ([P, i32, P, P, i32, i64, P, P, P, P, P, ctypes.POINTER(CacheStats)], i32),
+    "pmoe_cache_get_stats": ([P, ctypes.POINTER(CacheStats)], i32),
+    "pmoe_cache_resident_depth": ([P, i32, P], i32),
+    "pmoe_cache_eviction_log": ([P, P, i64, ctypes.POINTER(i64)], i32),
+    "pmoe_cache_destroy": ([P], i32),
+    "pmoe_cache_sim_independent": ([i32, i32, i64, i64, P, P, P, P, P, ctypes.POINTER(i64)], i32),
+    "pmoe_route_host": ([P, i32, i32, i32, P, P], i32),
+    "pmoe_residual_norm": ([P, P, i32, i32, P, P], i32),
 }
 
 for _name, (_args, _res) in _SIGS.items():
@@ -201,3 +219,95 @@ def materialise_layer_fwd(L: Layer, x, ids, w, depth, T, k, y, ws, ws_bytes, str
     _check("pmoe_materialise_layer_fwd", _lib.pmoe_materialise_layer_fwd(
         ctypes.byref(L), _ptr(x), _ptr(ids), _ptr(w), _ptr(depth), T, k, _ptr(y), _ptr(ws), ws_bytes,
         _stream(stream)))
+
+
+def route_host(logits, T, E, k, ids, w) -> None:
+    """pmoe_route on host arrays (numpy), synchronous."""
+    _check("pmoe_route_host", _lib.pmoe_route_host(_ptr(logits), T, E, k, _ptr(ids), _ptr(w)))
+
+
+def residual_norm(r, y, T, H, x, stream=None) -> None:
+    _check("pmoe_residual_norm", _lib.pmoe_residual_norm(_ptr(r), _ptr(y), T, H, _ptr(x), _stream(stream)))
+
+
+def _event(e):
+    if e is None:
+        return None
+    return e.cuda_event if hasattr(e, "cuda_event") else int(e)
+
+
+class Cache:
+    """pmoe_cache handle: the HBM prefix cache (host state in the library).
+
+    pool / page_table: device tensors the caller keeps alive (both None for a
+    host-only cache that only takes decisions)."""
+
+    def __init__(self, layers, experts, slots, slot_words, pool=None, page_table=None, keep_log=False):
+        h = P()
+        _check("pmoe_cache_create", _lib.pmoe_cache_create(layers, experts, slots, slot_words, _ptr(pool),
+                                                           _ptr(page_table), int(keep_log), ctypes.byref(h)))
+        self._h = h
+        self.layers, self.experts, self.slots, self.slot_words = layers, experts, slots, slot_words
+        self._host_ptrs = None
+
+    def set_host_planes(self, ptrs):
+        """ptrs: one pinned host pointer (int or tensor) per layer."""
+        arr = (P * self.layers)(*[_ptr(p) for p in ptrs])
+        self._host_ptrs = arr
+
+    def extend(self, layer, experts, need, batch, side=None, after=None, done=None, resident_before=None):
+        """experts: int32 numpy [n]; need: uint8 numpy [n]. Returns CacheStats (accumulated)."""
+        import numpy as np
+        experts = np.ascontiguousarray(experts, dtype=np.int32)
+        need = np.ascontiguousarray(need, dtype=np.uint8)
+        st = CacheStats()
+        _check("pmoe_cache_extend", _lib.pmoe_cache_extend(
+            self._h, layer, _ptr(experts), _ptr(need), len(experts), int(batch), self._host_ptrs,
+            _stream(side), _event(after), _event(done), _ptr(resident_before), ctypes.byref(st)))
+        return st
+
+    def stats(self):
+        st = CacheStats()
+        _check("pmoe_cache_get_stats", _lib.pmoe_cache_get_stats(self._h, ctypes.byref(st)))
+        return st
+
+    def resident_depth(self, layer):
+        import numpy as np
+        d = np.zeros(self.experts, dtype=np.uint8)
+        _check("pmoe_cache_resident_depth", _lib.pmoe_cache_resident_depth(self._h, layer, _ptr(d)))
+        return d
+
+    def eviction_log(self):
+        import numpy as np
+        n = i64(0)
+        _check("pmoe_cache_eviction_log", _lib.pmoe_cache_eviction_log(self._h, None, 0, ctypes.byref(n)))
+        out = np.zeros(max(n.value, 1), dtype=np.int64)
+        _check("pmoe_cache_eviction_log", _lib.pmoe_cache_eviction_log(self._h, _ptr(out), n.value,
+                                                                       ctypes.byref(n)))
+        return out[:n.value]
+
+    def close(self):
+        if self._h:
+            _check("pmoe_cache_destroy", _lib.pmoe_cache_destroy(self._h))
+            self._h = P()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def cache_sim_independent(layers, experts, cap_planes, layer, expert, need, batch):
+    """Independent-precision baseline on a trace: (hit uint8 [n], planes_fetched)."""
+    import numpy as np
+    layer = np.ascontiguousarray(layer, dtype=np.int32)
+    expert = np.ascontiguousarray(expert, dtype=np.int32)
+    need = np.ascontiguousarray(need, dtype=np.uint8)
+    batch = np.ascontiguousarray(batch, dtype=np.int64)
+    hit = np.zeros(len(layer), dtype=np.uint8)
+    fetched = i64(0)
+    _check("pmoe_cache_sim_independent", _lib.pmoe_cache_sim_independent(
+        layers, experts, cap_planes, len(layer), _ptr(layer), _ptr(expert), _ptr(need), _ptr(batch),
+        _ptr(hit), ctypes.byref(fetched)))
+    return hit, fetched.value

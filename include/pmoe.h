@@ -280,6 +280,125 @@ PMOE_API pmoe_status pmoe_materialise_layer_fwd(const pmoe_layer *L, const uint1
                                        const float *w, const uint8_t *depth, int T, int k,
                                        float *y, void *ws, size_t ws_bytes, pmoe_stream stream);
 
+/* ------------------------------------------------------------------ */
+/* Prefix cache [T#11, T#13, T#35, A: Abstract]                        */
+/* ------------------------------------------------------------------ */
+
+/*
+ * An HBM cache of expert prefixes for `layers` MoE layers of `experts`
+ * experts each, in a pool of plane slots (one slot = plane p of one expert,
+ * all three matrices, the pmoe_layer slot layout). Every (layer, expert) has
+ * one shared state whatever precision is asked of it [T#13]: its resident
+ * depth r (planes 0..r-1 in slots) and a last-use time per plane. An access
+ * (layer, expert, need b), time = its index since creation:
+ *   r >= b: hit, nothing copied; planes 0..b-1 take the current time;
+ *   r <  b: planes 0..r-1 take the current time; only the missing planes
+ *           r..b-1 are copied from host memory into free slots [T#35] and
+ *           take the current time; the depth becomes b.
+ * When no slot is free, the resident plane with the oldest time is evicted,
+ * which is always the deepest plane of its entry since a use refreshes a
+ * prefix (ties to the lowest layer*experts + expert); that entry's depth
+ * drops by one. Entries accessed in the current batch are never evicted.
+ *
+ * Memory (caller-owned, kept by the cache until destroyed):
+ *   pool: device uint32 [slots * slot_words]; slot s at pool + s*slot_words.
+ *   page_table: device int32 [layers][experts][8]: slot of plane p of expert
+ *     e of layer l, or -1. pmoe_layer.slot_of of layer l is
+ *     page_table + l*experts*8 (and pmoe_layer.pool = pool).
+ *   host planes of layer l (pmoe_cache_extend): pinned host uint32
+ *     [experts][8][slot_words]: plane p of expert e at (e*8 + p)*slot_words.
+ */
+typedef struct pmoe_cache pmoe_cache;
+
+typedef struct {
+    int64_t requests;       /* accesses */
+    int64_t hits;           /* accesses whose resident depth covered the need */
+    int64_t planes_fetched; /* expert-planes copied host -> device */
+    int64_t bytes_fetched;  /* their bytes */
+    int64_t planes_evicted;
+} pmoe_cache_stats;
+
+/*
+ * pmoe_cache_create: empty cache of `slots` slots of slot_words words
+ * (slot_words % 4 == 0). pool and page_table both NULL make a host-only
+ * cache: the same decisions and statistics, no data moved (planning and
+ * simulation). Otherwise the page table is set to -1 (synchronously).
+ * keep_log != 0 records every eviction (pmoe_cache_eviction_log).
+ * Allocates host memory only: the state, and a small mapped pinned area for
+ * page-table updates. layers*experts*8 and slots must fit in int32.
+ */
+PMOE_API pmoe_status pmoe_cache_create(int layers, int experts, int64_t slots, int64_t slot_words,
+                                       uint32_t *pool, int32_t *page_table, int keep_log, pmoe_cache **out);
+
+/*
+ * pmoe_cache_extend: applies the accesses (layer, experts[i], need[i]),
+ * i < n, in order, all in batch `batch` (the caller's id of the step whose
+ * kernels use them; an entry accessed in the current batch is pinned).
+ * Missing planes are copied with one cudaMemcpyAsync each on stream `side`
+ * from host_planes[layer] (host pointer array, indexed by layer; pinned
+ * memory), then the page-table entries of fetched and evicted planes are
+ * written by a small kernel on `side`, then `done` (may be NULL) is recorded
+ * on `side`. Kernels that read the pool must wait for `done`.
+ * Evicted slots are overwritten: if the call evicts and `after` is not NULL,
+ * `side` first waits for `after`, which the caller records on its compute
+ * stream after the last kernel of the previous batch.
+ *   experts: host int32 [n], need: host uint8 [n] in 1..8,
+ *   resident_before: host uint8 [n], the depth each access found (may be
+ *   NULL); stats: the cache's accumulated counters after the call (may be
+ *   NULL). Host-only caches ignore host_planes, side, after and done.
+ * Errors: PMOE_ERR_INVALID_ARG (nothing changed); PMOE_ERR_OUT_OF_SLOTS
+ * when the pinned entries of the batch leave no room (the accesses before
+ * the failing one are applied and their copies enqueued); PMOE_ERR_CUDA.
+ */
+PMOE_API pmoe_status pmoe_cache_extend(pmoe_cache *c, int layer, const int32_t *experts, const uint8_t *need,
+                                       int n, int64_t batch, const uint32_t *const *host_planes,
+                                       pmoe_stream side, pmoe_event after, pmoe_event done,
+                                       uint8_t *resident_before, pmoe_cache_stats *stats);
+
+/* Accumulated counters. */
+PMOE_API pmoe_status pmoe_cache_get_stats(const pmoe_cache *c, pmoe_cache_stats *stats);
+/* Resident depth of every expert of a layer: host uint8 [experts]. */
+PMOE_API pmoe_status pmoe_cache_resident_depth(const pmoe_cache *c, int layer, uint8_t *depth);
+/*
+ * Evictions so far, oldest first, as (layer*experts + expert)*8 + plane:
+ * up to cap written to log (host int64), the total count to *n.
+ * PMOE_ERR_UNSUPPORTED if the cache was created without keep_log.
+ */
+PMOE_API pmoe_status pmoe_cache_eviction_log(const pmoe_cache *c, int64_t *log, int64_t cap, int64_t *n);
+/* Frees the host state (waits for its pending page-table updates); the pool and page table stay the caller's. */
+PMOE_API pmoe_status pmoe_cache_destroy(pmoe_cache *c);
+
+/*
+ * pmoe_cache_sim_independent [T#11]: hit rate of the independent-precision
+ * design on an access trace, host only: every (layer, expert, bits) is its
+ * own object of `bits` planes; an access hits only if that exact object is
+ * resident; a miss loads all its planes and evicts whole least-recently-used
+ * objects (not those of the current batch) until it fits in cap_planes.
+ *   layer, expert: host int32 [n]; need: host uint8 [n]; batch: host int64
+ *   [n]; hit: host uint8 [n] out (1 hit, 0 miss); *planes_fetched out.
+ * PMOE_ERR_OUT_OF_SLOTS if an access cannot fit (outputs up to it written).
+ */
+PMOE_API pmoe_status pmoe_cache_sim_independent(int layers, int experts, int64_t cap_planes, int64_t n,
+                                                const int32_t *layer, const int32_t *expert,
+                                                const uint8_t *need, const int64_t *batch, uint8_t *hit,
+                                                int64_t *planes_fetched);
+
+/*
+ * pmoe_route_host: pmoe_route on host pointers (synchronous), for callers
+ * that plan cache top-ups before launching the layer: ids (ties to the lower
+ * id, larger logits first) and softmax weights in double rounded to float.
+ */
+PMOE_API pmoe_status pmoe_route_host(const float *logits, int T, int E, int k, int32_t *ids, float *w);
+
+/*
+ * pmoe_residual_norm: the residual stream between stacked layers, per token
+ * t: r_t += y_t (skipped when y is NULL), then x_t = bf16(r_t * (1/rms(r_t)))
+ * with rms = sqrt(mean of r_t^2) (x_t = 0 when rms is 0). Deterministic
+ * (fixed-order float sums). r: device float [T*H] (updated), y: device float
+ * [T*H] or NULL, x: device bf16 [T*H] out. H % 4 == 0.
+ */
+PMOE_API pmoe_status pmoe_residual_norm(float *r, const float *y, int T, int H, uint16_t *x, pmoe_stream stream);
+
 #ifdef __cplusplus
 }
 #endif
