@@ -47,6 +47,11 @@ def parse():
     # a smaller layer of the same shape (fewer experts) and fewer distinct tokens, for profiler captures
     ap.add_argument("--experts", type=int, default=E)
     ap.add_argument("--tokens", type=int, default=1024)
+    # the stacked-layer decode through the HBM prefix cache (pinned host planes, side-stream top-ups)
+    ap.add_argument("--workload", default="layer", choices=["layer", "cache"])
+    ap.add_argument("--layers", type=int, default=16)
+    ap.add_argument("--cache-tokens", type=int, default=256)
+    ap.add_argument("--cache-frac", type=float, default=0.4)
     return ap.parse_args()
 
 
@@ -231,6 +236,125 @@ def reference_arm(args):
     return 0
 
 
+# ----------------------------------------------------------------------------- cached stack
+
+def host_mem_available():
+    try:
+        with open("/proc/meminfo") as f:
+            for line in f:
+                if line.startswith("MemAvailable:"):
+                    return int(line.split()[1]) * 1024
+    except OSError:
+        pass
+    return 0
+
+
+def cache_bench(args):
+    """Stacked layers of the 512-expert shape decoding sequential batch-1 tokens through the HBM
+    prefix cache from a cold start: router logits AR(1) (rho 0.8) per layer, cache capped at a
+    fraction of all layers' 8-plane bytes. Host planes are pinned; when host memory cannot hold a
+    copy per layer, layers share backing planes (layer l uses backing l % n) while staying
+    distinct cache entries."""
+    import numpy as np
+    import torch
+
+    import __graft_entry__
+    __graft_entry__.build()
+    import bitplane_mixed_precision_b200 as pm
+    import synth
+    from bitplane_mixed_precision_b200.cached import CachedStack
+    from bitplane_mixed_precision_b200.store import ResidentLayer
+
+    Lr, T = args.layers, args.cache_tokens
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    st = torch.cuda.current_stream(dev)
+    slot_bytes = 3 * H * I // 8
+    per_backing = E * 8 * slot_bytes
+    avail = host_mem_available()
+    n_back = max(1, min(Lr, int(0.6 * avail // per_backing)))
+    slots = int(args.cache_frac * Lr * E * 8)
+
+    def make(b):
+        def fill(e, m, w):
+            synth.expert_weights_device(SEED, b, e, m, w.numel(), w.data_ptr(), st.cuda_stream)
+        R = ResidentLayer(E, H, I, G, fill, device=dev)
+        torch.cuda.synchronize()
+        return R
+
+    t0 = time.perf_counter()
+    sens = [synth.sensitivities(SEED, b, E) for b in range(n_back)]
+    S = CachedStack(Lr, E, H, I, G, K_TOP, AVG, slots, (n_back, make), sens, device=dev)
+    torch.cuda.empty_cache()
+    setup_s = time.perf_counter() - t0
+    logits = np.stack([synth.ar1_logits(SEED, l, T, E) for l in range(Lr)], axis=1)
+    emb = torch.from_numpy(np.stack([synth.activation_f32(SEED, t, 99, H) for t in range(T)])).pin_memory()
+    r = torch.empty(H, dtype=torch.float32, device=dev)
+    x = torch.empty(H, dtype=torch.int16, device=dev)
+    y = torch.empty(H, dtype=torch.float32, device=dev)
+    y_last = torch.empty(T, H, dtype=torch.float32, device=dev)
+    y_host = torch.empty(T, H, dtype=torch.float32).pin_memory()
+    marks = []
+    torch.cuda.synchronize()
+    t_start = time.perf_counter()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for t in range(T):
+        r.copy_(emb[t], non_blocking=True)
+        pm.residual_norm(r, None, 1, H, x, st)
+        S.decode_token(logits[t], r, x, y, t, stream=st)
+        y_last[t].copy_(y)
+        y_host[t].copy_(y, non_blocking=True)
+        if t == T // 2:
+            torch.cuda.synchronize()
+            marks.append((time.perf_counter(), S.cache.stats().as_dict()))
+    e1.record(st)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t_start
+    dev_s = e0.elapsed_time(e1) * 1e-3
+    err = S.check_errors()
+    stats = S.cache.stats().as_dict()
+    lay, exp_, dep, bat = S.trace_arrays()
+    hit_i, fetched_i = pm.cache_sim_independent(Lr, E, slots, lay, exp_, dep, bat)
+    req_planes = int(dep.sum())
+    t_half, st_half = marks[0]
+    warm_tokens = T - (T // 2 + 1)           # tokens after the mid-run synchronisation
+    warm_s = wall - (t_half - t_start)
+    S.close()
+    line = {
+        "metric": "cached stacked-layer decode tokens/s (HBM prefix cache over pinned host planes)",
+        "value": T / wall, "unit": "tokens/s", "n_gpus": 1, "steps": T, "warmup": 0,
+        "ms_per_step": wall * 1e3 / T, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "s8 mma / s32 acc / f32", "data": "synthetic",
+        "config": {"workload": f"cached_decode_l{Lr}_e{E}_top10_h4096_i1024_g128_avg2.5_batch1",
+                   "layers": Lr, "experts": E, "tokens": T, "cache_slots": slots,
+                   "cache_bytes": slots * slot_bytes, "cache_frac": args.cache_frac,
+                   "host_backing_layers": n_back, "host_mem_available": avail,
+                   "logits": "AR(1) rho 0.8 per layer", "start": "cold"},
+        "layer_tokens_per_s": T * Lr / wall,
+        "steady_tokens_per_s": warm_tokens / warm_s if warm_s > 0 else None,
+        "device_s": dev_s, "wall_s": wall, "setup_s": setup_s,
+        "cache": {
+            "requests": stats["requests"], "prefix_hit_rate": stats["hits"] / max(stats["requests"], 1),
+            "independent_hit_rate": float(hit_i.mean()),
+            "prefix_planes_fetched": stats["planes_fetched"], "independent_planes_fetched": fetched_i,
+            "planes_requested": req_planes,
+            "prefix_byte_hit_rate": 1.0 - stats["planes_fetched"] / max(req_planes, 1),
+            "independent_byte_hit_rate": 1.0 - fetched_i / max(req_planes, 1),
+            "h2d_bytes_per_token": stats["bytes_fetched"] / T,
+            "h2d_gbs": stats["bytes_fetched"] / wall / 1e9,
+            "planes_evicted": stats["planes_evicted"],
+            "second_half_prefix_hit_rate": (stats["hits"] - st_half["hits"]) /
+                                           max(stats["requests"] - st_half["requests"], 1),
+        },
+        "layer_error": list(err),
+        "gpu_launches": T * (Lr * 3 + 1),  # per layer prep + expert kernel + residual; plus page-table updates
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # ----------------------------------------------------------------------------- GPU arm
 
 def main():
@@ -239,6 +363,8 @@ def main():
     E, N_TOKENS = args.experts, args.tokens
     if args.impl == "reference":
         return reference_arm(args)
+    if args.workload == "cache":
+        return cache_bench(args)
 
     import numpy as np
     import torch
@@ -386,6 +512,49 @@ def main():
         del g
     graphs.clear()
 
+    # the same tokens (routing recorded above) through pmoe_moe_layer_fwd: at the selected depths,
+    # at a uniform 4 bits, and through the materialise-to-bf16 ablation; graph-captured, 256 tokens
+    nv = min(256, N_TOKENS)
+    dep4 = torch.full((N_TOKENS, K_TOP), 4, dtype=torch.uint8, device=dev)
+    mws_bytes = pm.materialise_workspace_bytes(T, K_TOP, E, H, I)
+    mws = torch.empty(mws_bytes, dtype=torch.uint8, device=dev)
+
+    def variant(call):
+        for i in range(4):
+            call(i, stream)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            for i in range(nv):
+                call(i, cap)
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        del g
+        return a.elapsed_time(b) * 1e-3 / nv
+
+    t_sel = variant(lambda i, st: pm.moe_layer_fwd(R.layer, x[i], ids[i], wts[i], dep[i], T, K_TOP, y[i], ws,
+                                                   ws_bytes, st))
+    t_u4 = variant(lambda i, st: pm.moe_layer_fwd(R.layer, x[i], ids[i], wts[i], dep4[i], T, K_TOP, y[i], ws,
+                                                  ws_bytes, st))
+    t_mat = variant(lambda i, st: pm.materialise_layer_fwd(R.layer, x[i], ids[i], wts[i], dep[i], T, K_TOP,
+                                                           y[i], mws, mws_bytes, st))
+    del mws
+    sel_planes = float(dep_h[:nv].sum(axis=1).mean()) * 3 * PLANE_BYTES
+    variants = {
+        "tokens": nv,
+        "layer_fwd_selected_depths": {"tokens_per_s": 1.0 / t_sel, "us_per_token": t_sel * 1e6,
+                                      "bitplane_gbs": sel_planes / t_sel / 1e9},
+        "uniform_b4": {"tokens_per_s": 1.0 / t_u4, "us_per_token": t_u4 * 1e6,
+                       "bitplane_gbs": K_TOP * 4 * 3 * PLANE_BYTES / t_u4 / 1e9},
+        "materialise_bf16_ablation": {"tokens_per_s": 1.0 / t_mat, "us_per_token": t_mat * 1e6,
+                                      "direct_speedup": t_mat / t_sel},
+    }
+
     if rank == 0:
         pk, pk_kind = peaks()
         peak = float(pk["hbm_gbs"])
@@ -410,7 +579,7 @@ def main():
             "bitplane_gbs": bitplane_gbs, "bitplane_frac_of_8000": bitplane_gbs / 8000.0,
             "expert_kernels_us": 1e6 * sum(kdur) / len(kdur),
             "mean_bits": float(dep_h.mean()),
-            "cpu_baseline": cpu, "e2e": e2e,
+            "cpu_baseline": cpu, "e2e": e2e, "variants": variants,
             "gpu_launches": kernels_per_step * args.steps,
             "clocks": clk,
         }

@@ -64,6 +64,7 @@ struct pmoe_cache {
     bool keep_log = false;
 
     std::vector<int32_t> pt;        // host mirror [L*E*8]
+    std::vector<unsigned char> dirty; // [L*E*8]: entry changed in the current call
     std::vector<uint8_t> depth;     // [L*E]
     std::vector<int64_t> ts;        // [L*E*8] last use of each plane
     std::vector<int64_t> last_batch; // [L*E]: batch of the last access (meaningful while resident)
@@ -145,6 +146,7 @@ pmoe_status pmoe_cache_create(int layers, int experts, int64_t slots, int64_t sl
     c->keep_log = keep_log != 0;
     try {
         c->pt.assign((size_t)NE * 8, -1);
+        c->dirty.assign((size_t)NE * 8, 0);
         c->depth.assign((size_t)NE, 0);
         c->ts.assign((size_t)NE * 8, 0);
         c->last_batch.assign((size_t)NE, 0);
@@ -204,7 +206,13 @@ pmoe_status pmoe_cache_extend(pmoe_cache *c, int layer, const int32_t *experts, 
         src = host_planes[layer];
     }
     cudaStream_t st = (cudaStream_t)side;
-    std::vector<int2> upd;
+    std::vector<int> touched; // page-table entries changed by this call (each once)
+    auto touch = [&](size_t k) {
+        if (moves && !c->dirty[k]) {
+            c->dirty[k] = 1;
+            touched.push_back((int)k);
+        }
+    };
     struct Copy {
         int32_t slot;
         int64_t from; // word offset in the layer's host planes
@@ -249,8 +257,7 @@ pmoe_status pmoe_cache_extend(pmoe_cache *c, int layer, const int32_t *experts, 
             const size_t k = (size_t)y * 8 + p;
             c->free_slots.push_back(c->pt[k]);
             c->pt[k] = -1;
-            if (moves)
-                upd.push_back(make_int2((int)k, -1));
+            touch(k);
             c->used -= 1;
             c->stats.planes_evicted += 1;
             if (c->keep_log)
@@ -270,10 +277,9 @@ pmoe_status pmoe_cache_extend(pmoe_cache *c, int layer, const int32_t *experts, 
             const size_t k = (size_t)x * 8 + p;
             c->pt[k] = s;
             c->ts[k] = now;
-            if (moves) {
-                upd.push_back(make_int2((int)k, s));
+            touch(k);
+            if (moves)
                 copies.push_back({s, ((int64_t)e * 8 + p) * c->slot_words});
-            }
         }
         c->depth[(size_t)x] = (uint8_t)b;
         c->used += want;
@@ -282,6 +288,13 @@ pmoe_status pmoe_cache_extend(pmoe_cache *c, int layer, const int32_t *experts, 
         c->order.insert({c->deepest_ts(x), x});
     }
 
+    // an entry evicted and fetched again in one call is written once, with its final slot
+    std::vector<int2> upd;
+    upd.reserve(touched.size());
+    for (int k : touched) {
+        upd.push_back(make_int2(k, c->pt[(size_t)k]));
+        c->dirty[(size_t)k] = 0;
+    }
     if (moves && (!copies.empty() || !upd.empty())) {
         if (evicted && after)
             PMOE_CUDA(cudaStreamWaitEvent(st, (cudaEvent_t)after, 0));

@@ -247,7 +247,9 @@ __device__ void gateup_tile_done(const LayerWs &W, int I, int u, int s32, int bl
 }
 
 // After a pair's 128 output rows are written: the last of the token's k pairs
-// sums them into y in slot order.
+// sums them into y in slot order. Lane owns rows lane + 32*i (i < 4); the
+// partial rows of 4 slots at a time are loaded before they are summed, so the
+// L2 round trips overlap instead of following one another.
 __device__ void down_rows_done(const Args &a, int pair, int s128)
 {
     const LayerWs &W = a.W;
@@ -261,12 +263,29 @@ __device__ void down_rows_done(const Args &a, int pair, int s128)
     __syncwarp();
     if (!last)
         return;
-    for (int r = lane; r < 128; r += 32) {
-        float s = 0.0f;
-        for (int i = 0; i < k; ++i)
-            s = __fmaf_rn(__ldg(a.wts + tok * k + i), __ldcg(W.part + (int64_t)(tok * k + i) * H + 128 * s128 + r), s);
-        a.y[(int64_t)tok * H + 128 * s128 + r] = s;
+    const float *part = W.part + (int64_t)tok * k * H + 128 * s128 + lane;
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    for (int i0 = 0; i0 < k; i0 += 4) {
+        float v[4][4], wt[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const bool ok = i0 + j < k;
+            wt[j] = ok ? __ldg(a.wts + tok * k + i0 + j) : 0.0f;
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+                v[j][r] = ok ? __ldcg(part + (int64_t)(i0 + j) * H + 32 * r) : 0.0f;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (i0 + j < k) {
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+                    acc[r] = __fmaf_rn(wt[j], v[j][r], acc[r]);
+            }
     }
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+        a.y[(int64_t)tok * H + 128 * s128 + 32 * r + lane] = acc[r];
 }
 
 template <int GS>
@@ -326,6 +345,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
             }
         };
         while (ok) {
+            // claim only once the queue has room: an item is taken when this SM can start on it soon
+            const int qs = qi % QDEPTH;
+            if (qi >= QDEPTH && !pipe::mbar_wait(&S.qempty[qs], ((qi / QDEPTH) + 1) & 1, deadline)) {
+                set_error(W, kErrTimeout, 1);
+                break;
+            }
             Desc d;
             const int u = atomicAdd(&W.flags[kFlagSched], 1);
             if (u >= total) {
@@ -341,11 +366,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                 d.strip = (u - totalA) % SB;
             }
             d.c0 = c;
-            const int qs = qi % QDEPTH;
-            if (qi >= QDEPTH && !pipe::mbar_wait(&S.qempty[qs], ((qi / QDEPTH) + 1) & 1, deadline)) {
-                set_error(W, kErrTimeout, 1);
-                break;
-            }
             S.q[qs] = d;
             pipe::mbar_arrive(&S.qfull[qs]);
             ++qi;

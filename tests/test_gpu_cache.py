@@ -1,0 +1,138 @@
+"""Cached decode on the GPU: stacked layers whose planes come from pinned host
+memory through the prefix cache give the same outputs, bit for bit, as the
+same layers fully resident in HBM (PagedMoE transcript cues 13, 35: a cached
+prefix is the same data as the stored expert); the cache's decisions on the
+run's own access trace equal the oracle simulator's; the decode's first
+layer also matches the oracle within the layer tolerance."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_common import assert_close
+
+pytestmark = pytest.mark.gpu
+
+L, E, H, I, G, K, AVG = 3, 16, 1024, 256, 128, 4, 2.5
+SEED = 404
+
+
+def _backing(synth_mod, b, dev):
+    from bitplane_mixed_precision_b200.store import ResidentLayer
+    st = torch.cuda.current_stream(dev)
+
+    def fill(e, m, w):
+        synth_mod.expert_weights_device(SEED, b, e, m, w.numel(), w.data_ptr(), st.cuda_stream)
+    return ResidentLayer(E, H, I, G, fill, device=dev)
+
+
+@pytest.fixture(scope="module")
+def stack_setup(synth_mod):
+    synth_mod.build()  # the device generator fills the experts
+    dev = torch.device("cuda", 0)
+    backs = [_backing(synth_mod, b, dev) for b in range(2)]  # layers 0 and 2 share backing 0
+    sens = [synth_mod.sensitivities(SEED, b, E) for b in range(2)]
+    torch.cuda.synchronize()
+    return dev, backs, sens
+
+
+def _run(stack_setup, synth_mod, slots, tokens, keep_log=True):
+    import bitplane_mixed_precision_b200 as pm
+    from bitplane_mixed_precision_b200.cached import CachedStack
+    dev, backs, sens = stack_setup
+    S = CachedStack(L, E, H, I, G, K, AVG, slots, backs, sens, device=dev, keep_log=keep_log)
+    logits = np.stack([synth_mod.ar1_logits(SEED, l, tokens, E) for l in range(L)], axis=1)  # [t, l, E]
+    emb = [synth_mod.activation_f32(SEED, t, 99, H) for t in range(tokens)]
+    r = torch.empty(H, dtype=torch.float32, device=dev)
+    x = torch.empty(H, dtype=torch.int16, device=dev)
+    y = torch.empty(H, dtype=torch.float32, device=dev)
+    # resident reference: same layers, every plane in its own slot
+    rr = torch.empty_like(r)
+    xr = torch.empty_like(x)
+    yr = torch.empty_like(y)
+    ws = torch.empty(pm.layer_workspace_bytes(1, K, E, H, I), dtype=torch.uint8, device=dev)
+    outs, refs, routes, xs = [], [], [], []
+    for t in range(tokens):
+        r.copy_(torch.from_numpy(emb[t]))
+        pm.residual_norm(r, None, 1, H, x)
+        rr.copy_(r)
+        xr.copy_(x)
+        xs.append(x.clone())
+        y_out = torch.empty(L, H, dtype=torch.float32, device=dev)
+        s = S.decode_token(logits[t], r, x, y, t, y_out=y_out)
+        ids, w, dep = S.routing(s)
+        routes.append((ids, w, dep))
+        y_ref = torch.empty(L, H, dtype=torch.float32, device=dev)
+        for l in range(L):
+            idd = torch.from_numpy(ids[l]).to(dev)
+            wd = torch.from_numpy(w[l]).to(dev)
+            dd = torch.from_numpy(dep[l]).to(dev)
+            pm.moe_layer_fwd(backs[l % 2].layer, xr, idd, wd, dd, 1, K, yr, ws, ws.numel())
+            y_ref[l].copy_(yr)
+            pm.residual_norm(rr, yr, 1, H, xr)
+        torch.cuda.synchronize()
+        assert S.check_errors() == (0, 0)
+        outs.append(y_out.cpu())
+        refs.append(y_ref.cpu())
+    return S, outs, refs, routes, logits, xs
+
+
+def test_cached_equals_resident_bitwise(stack_setup, synth_mod, oracle_mod):
+    # 48 slots of 3*16*8 = 384: evictions on most tokens; a token pins <= 3 layers x 10 planes
+    S, outs, refs, routes, logits, _ = _run(stack_setup, synth_mod, slots=48, tokens=12)
+    for t, (a, b) in enumerate(zip(outs, refs)):
+        assert torch.equal(a, b), f"token {t}"
+    st = S.cache.stats()
+    assert st.planes_evicted > 0 and st.hits > 0
+    lay, exp_, dep, bat = S.trace_arrays()
+    before_o, log_o, fetched_o = oracle_mod.cache_sim_prefix(L, E, 48, lay.astype(np.int32),
+                                                             exp_.astype(np.int32), dep.astype(np.uint8),
+                                                             bat.astype(np.int32))
+    assert np.array_equal(S.cache.eviction_log(), log_o)
+    assert st.planes_fetched == fetched_o
+    assert st.bytes_fetched == fetched_o * S.slot_words * 4
+    S.close()
+
+
+def test_cached_routing_matches_oracle(stack_setup, synth_mod, oracle_mod):
+    S, outs, refs, routes, logits, xs = _run(stack_setup, synth_mod, slots=64, tokens=3)
+    dev, backs, sens = stack_setup
+    for t in range(3):
+        for l in range(L):
+            ids, w, dep = routes[t]
+            ids_o, w_o = oracle_mod.route(logits[t][l][None, :], K)
+            assert np.array_equal(ids[l], ids_o[0]) and np.array_equal(w[l], w_o[0])
+            dep_o = oracle_mod.select(w[l][None, :], ids[l][None, :], sens[l % 2], AVG)
+            assert np.array_equal(dep[l], dep_o[0])
+    S.close()
+
+
+def test_first_layer_matches_oracle(stack_setup, synth_mod):
+    from gpu_common import OracleExperts
+    import synth
+    dev, backs, sens = stack_setup
+    S, outs, refs, routes, logits, xs = _run(stack_setup, synth_mod, slots=64, tokens=2)
+    ox = OracleExperts(SEED, H, I, G, layer=0)
+    for t in range(2):
+        ids, w, dep = routes[t]
+        x64 = synth.bf16_to_f32(xs[t].cpu().numpy().view(np.uint16)).astype(np.float64)
+        y_o = ox.run(E, ids[:1], w[:1], dep[:1], x64[None, :])
+        assert_close(outs[t][0].numpy()[None, :], y_o)
+    S.close()
+
+
+def test_residual_norm_matches_numpy(stack_setup):
+    import bitplane_mixed_precision_b200 as pm
+    dev = stack_setup[0]
+    g = torch.Generator().manual_seed(3)
+    T, Hh = 3, 1024
+    r = torch.randn(T, Hh, generator=g)
+    y = torch.randn(T, Hh, generator=g)
+    rd, yd = r.to(dev), y.to(dev)
+    x = torch.empty(T, Hh, dtype=torch.int16, device=dev)
+    pm.residual_norm(rd, yd, T, Hh, x)
+    torch.cuda.synchronize()
+    r2 = (r + y).numpy().astype(np.float64)
+    assert np.array_equal(rd.cpu().numpy(), (r + y).numpy())
+    xf = (x.cpu().numpy().astype(np.int32) << 16).astype(np.uint32).view(np.float32)
+    ref = r2 / np.sqrt((r2 ** 2).mean(axis=1, keepdims=True))
+    assert np.max(np.abs(xf - ref)) <= 2 ** -7 * np.max(np.abs(ref))
