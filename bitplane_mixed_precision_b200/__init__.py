@@ -16,7 +16,7 @@ LIB_PATH = os.path.join(_HERE, "libpmoe.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"libpmoe.so is missing at {LIB_PATH}; build it with "
-                      "`python -m bitplane_mixed_precision_b200.build`")
+                      "`python bitplane_mixed_precision_b200/build.py` or __graft_entry__.build()")
 
 _lib = ctypes.CDLL(LIB_PATH)
 

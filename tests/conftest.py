@@ -12,6 +12,12 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
 
 
+def pytest_sessionstart(session):
+    # the test modules import the binding, which needs the library: build it (or find it current)
+    import __graft_entry__
+    __graft_entry__._library_builder().build()
+
+
 def has_gpu() -> bool:
     try:
         import torch

@@ -12,8 +12,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def pm():
-    from bitplane_mixed_precision_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__._library_builder().build()
     import bitplane_mixed_precision_b200 as pm
     return pm
 
