@@ -429,7 +429,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                                 set_error(W, kErrTimeout, 5);
                                 break;
                             }
-                            __nanosleep(32);
+                            __nanosleep(256);
                         }
                         pipe::fence_proxy_async();
                     }
@@ -602,7 +602,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                         fine = false;
                         break;
                     }
-                    __nanosleep(32);
+                    __nanosleep(256);
                 }
             }
             fine = __shfl_sync(0xffffffffu, (int)fine, 0) != 0;

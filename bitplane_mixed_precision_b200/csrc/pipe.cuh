@@ -44,14 +44,19 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  : "memory");
 }
 
+// Tests the phase with the given parity; if it is not complete the thread may
+// sleep until it completes, for at most kSuspendNs (so that waiting warps do
+// not take issue slots from the warps that compute).
+constexpr uint32_t kSuspendNs = 20000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 {
     uint32_t ok;
     asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+                 "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
                  "selp.u32 %0, 1, 0, p;\n\t}"
                  : "=r"(ok)
-                 : "r"(smem_u32(bar)), "r"(parity)
+                 : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
                  : "memory");
     return ok != 0;
 }
@@ -60,10 +65,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 // deadline (global timer, ns) passed first.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t deadline)
 {
-    for (uint32_t n = 1;; ++n) {
+    for (;;) {
         if (mbar_try_wait(bar, parity))
             return true;
-        if ((n & 15u) == 0 && globaltimer() > deadline)
+        if (globaltimer() > deadline)
             return false;
     }
 }
