@@ -210,6 +210,26 @@ __device__ __forceinline__ void decode_kstep(const uint32_t (&w)[8][2], int s, c
     }
 }
 
+// Depth 1 with an antisymmetric table (C[1][0] = -C[1][1], as for the Gaussian
+// tree): the value is C[1][1] * (2*bit - 1), so the A bytes are the signs +-1
+// themselves and one MMA per k-step suffices (no high/low split). The plane
+// word is masked to the t-word's bit of each nibble (bit r); r = 3 is moved to
+// bit 2, because a selector nibble with bit 3 set asks prmt for a sign fill.
+// Byte table: selector 0 -> -1, selector 1, 2 or 4 -> +1.
+__device__ __forceinline__ void decode_kstep_sign(const uint32_t (&w)[8][2], int s, uint32_t (&a)[4])
+{
+    constexpr uint32_t kLo = 0x000101FFu, kHi = 0x00000001u;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int q = 2 * s + u, h = q >> 2, r = q & 3;
+        uint32_t t = w[0][h] & (0x11111111u << r);
+        if (r == 3)
+            t >>= 1;
+        a[u] = prmt(kLo, kHi, t);
+        a[2 + u] = prmt(kLo, kHi, t >> 16);
+    }
+}
+
 // Prefix index (b bits, MSB first) of every weight of the lane's tile, in the
 // A-fragment order: out[q][j] for t-word q, nibble j.
 template <int B>

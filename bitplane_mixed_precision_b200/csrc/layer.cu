@@ -250,8 +250,16 @@ __global__ void __launch_bounds__(kPrepThreads) layer_prep_kernel(PrepArgs a)
             dst[r] = r == 0 ? tab.h[0] : r == 1 ? tab.h[1] : r == 2 ? tab.h[2] : tab.h[3];
             dst[4 + r] = r == 0 ? tab.l[0] : r == 1 ? tab.l[1] : r == 2 ? tab.l[2] : tab.l[3];
         }
-        if (lane == 0)
+        if (lane == 0) {
             dst[8] = (uint32_t)tab.f;
+            if (d == 1) {
+                // depth 1 of an antisymmetric table decodes to signs (see dev::decode_kstep_sign)
+                const float *cb = a.L.codebooks + ((int64_t)e * 3 + m) * 510;
+                const float c0 = __ldg(cb), c1 = __ldg(cb + 1);
+                dst[9] = __float_as_uint(c1);
+                dst[10] = (c0 == -c1) ? 1u : 0u;
+            }
+        }
     }
 }
 

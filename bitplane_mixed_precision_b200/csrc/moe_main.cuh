@@ -180,6 +180,44 @@ __device__ __forceinline__ void warp_block(const unsigned char *const (&pp)[8], 
     }
 }
 
+// Depth 1 of an antisymmetric table: +-1 bytes, one MMA per k-step, and the
+// group sums scaled by C[1][1] (table head word 9).
+template <int GS, int FRAG>
+__device__ __forceinline__ void warp_block_sign(const unsigned char *const (&pp)[8], int ntiles, int Q0,
+                                                const unsigned char *tabs, const uint32_t *fptr, int fstep,
+                                                const int *exps, const float *sc0, const float *sc1, float &acc0,
+                                                float &acc1)
+{
+    constexpr int NG = 4 / GS;
+    const float c1 = __uint_as_float(reinterpret_cast<const uint32_t *>(tabs)[9]);
+    const bool epi = exps != nullptr;
+    for (int j = 0; j < ntiles; ++j) {
+        uint32_t w[8][2];
+        const uint2 v = *reinterpret_cast<const uint2 *>(pp[0] + j * 256);
+        w[0][0] = v.x;
+        w[0][1] = v.y;
+        const float fac = epi ? c1 * pow2neg(exp_at<FRAG>(exps + Q0 + j)) : 0.0f;
+        int dh[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            uint32_t a[4];
+            dev::decode_kstep_sign(w, s, a);
+            uint2 bv = make_uint2(0u, 0u);
+            if (FRAG == 0 || fptr != nullptr)
+                bv = frag_at<FRAG>(fptr + (j * 4 + s) * fstep);
+            dev::mma_s8(dh, a, bv.x, bv.y);
+            if ((s + 1) % GS == 0) {
+                const int gi = j * NG + s / GS;
+                acc0 = __fmaf_rn((float)(dh[0] * 256 + dh[1]), sc0[gi] * fac, acc0);
+                acc1 = __fmaf_rn((float)(dh[2] * 256 + dh[3]), sc1[gi] * fac, acc1);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dh[i] = 0;
+            }
+        }
+    }
+}
+
 template <int GS, int FRAG>
 __device__ __forceinline__ void warp_block_any(int d, const unsigned char *const (&pp)[8], int ntiles, int Q0,
                                                const unsigned char *tabs, const uint32_t *big, const uint32_t *fptr,
@@ -187,7 +225,12 @@ __device__ __forceinline__ void warp_block_any(int d, const unsigned char *const
                                                float &acc0, float &acc1)
 {
     switch (d) {
-    case 1: warp_block<1, GS, FRAG>(pp, ntiles, Q0, tabs, big, fptr, fstep, exps, sc0, sc1, acc0, acc1); break;
+    case 1:
+        if (reinterpret_cast<const uint32_t *>(tabs)[10] != 0u)
+            warp_block_sign<GS, FRAG>(pp, ntiles, Q0, tabs, fptr, fstep, exps, sc0, sc1, acc0, acc1);
+        else
+            warp_block<1, GS, FRAG>(pp, ntiles, Q0, tabs, big, fptr, fstep, exps, sc0, sc1, acc0, acc1);
+        break;
     case 2: warp_block<2, GS, FRAG>(pp, ntiles, Q0, tabs, big, fptr, fstep, exps, sc0, sc1, acc0, acc1); break;
     case 3: warp_block<3, GS, FRAG>(pp, ntiles, Q0, tabs, big, fptr, fstep, exps, sc0, sc1, acc0, acc1); break;
     case 4: warp_block<4, GS, FRAG>(pp, ntiles, Q0, tabs, big, fptr, fstep, exps, sc0, sc1, acc0, acc1); break;
