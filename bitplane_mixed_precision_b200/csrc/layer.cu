@@ -47,7 +47,7 @@ LayerWs carve_layer_ws(void *ws, int T, int k, int H, int I, size_t *bytes)
     const size_t o_flags = take(64 * 4);
     const size_t o_bd = take(P * 4), o_bn = take(P * 4), o_bp = take(P * 16), o_be = take(P * 4);
     const size_t o_ue = take(P * 4), o_u0 = take(P * 4), o_un = take(P * 4), o_ub = take(P * 4);
-    const size_t o_ca = take(P * (I / 32) * 4), o_ch = take(P * (I / 128) * 4), o_rb = take(P * 4);
+    const size_t o_ca = take(P * (I / 16) * 4), o_ch = take(P * (I / 128) * 4), o_rb = take(P * 4);
     const size_t o_cb = take(P * (H / 128) * 4), o_yc = take((size_t)T * (H / 128) * 4);
     const size_t o_pa = take(P * (size_t)(I / 16) * 8 * 32 * 4), o_pb = take(P * (size_t)(H / 16) * 2 * 16 * 4);
     const size_t o_tab = take(P * 3 * kTabWords * 4);
@@ -162,7 +162,7 @@ __global__ void __launch_bounds__(kPrepThreads) layer_prep_kernel(PrepArgs a)
             }
         }
         const int ti = tid - 32 * n_rw, nt = 32 * nw;
-        for (int i = ti; i < P * (I / 32); i += nt)
+        for (int i = ti; i < P * (I / 16); i += nt)
             W.cntA[i] = 0;
         for (int i = ti; i < P * (I / 128); i += nt)
             W.cntH[i] = 0;
@@ -291,8 +291,9 @@ pmoe_status check_layer(const pmoe_layer *L, int T, int k)
         return PMOE_ERR_INVALID_ARG;
     if (T < 0 || k < 1 || k > 32 || k > L->E || (int64_t)T * k > kMaxPairs)
         return PMOE_ERR_INVALID_ARG;
-    // shapes the persistent kernel tiles: 8 warps share a 16-row strip of gate/up (H/128 tiles),
-    // 2 warps a strip of down (I/128 tiles); a ring slot holds 32 rows of H or 128 rows of I.
+    // shapes the persistent kernel tiles: 8 warps share each matrix of a 16-row gate/up item
+    // (H/128 tiles), 2 warps a 16-row strip of down (I/128 tiles); a ring slot holds the 16
+    // gate and 16 up rows of one plane, or 128 down rows of one plane.
     if (L->H % 1024 || L->H > 4096 || L->I % 256 || L->I > 1024)
         return PMOE_ERR_UNSUPPORTED;
     // an item's scale rows and table heads travel in one ring slot

@@ -32,8 +32,8 @@ struct LayerWs {
     int *blk_pair;   //   [4] pair index t*k + i of each member
     int *blk_expert; //   expert
     int *unit_expert, *unit_blk0, *unit_nblk, *unit_bmax; // per unit (one expert, <= 4 blocks)
-    int *cntA;       // per gate/up item (unit, 32 rows of I): consumer warps finished
-    int *cntH;       // per (unit, 128 rows of I): gate/up items finished
+    int *cntA;       // per gate/up item (unit, 16 rows of I): consumer warps finished
+    int *cntH;       // per (unit, 128 rows of I): gate/up items finished (8 per tile)
     int *readyB;     // per unit: 128-row tiles of h turned into fragments
     int *cntB;       // per down item (unit, 128 rows of H): consumer warps finished
     int *ycnt;       // [T][H/128]: pairs of a token whose down rows are written

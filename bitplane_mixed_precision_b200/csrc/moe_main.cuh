@@ -3,16 +3,19 @@
 // One CTA per SM: warp NCW is the producer, warps 0..NCW-1 consume.
 //
 // Producer: takes work items from a global counter (gate/up items first, then
-// down items; units deepest first), publishes each item in a small queue and
-// streams the item's bytes into a ring of 16 KB shared-memory slots with 1-D
-// bulk copies completing on mbarriers: one chunk per (matrix, plane) and a
-// "meta" chunk (the scale rows of the item's matrices and the decode tables of
-// its column blocks), ordered [gate planes | meta | up planes] or
-// [meta | down planes] so that no copy of an item ever waits for a slot the
-// same item still holds.
+// down items; units deepest first), one at a time once the two-entry item
+// queue has room, publishes each item in that queue and streams the item's
+// bytes into a ring of 16 KB shared-memory slots with 1-D bulk copies
+// completing on mbarriers: one chunk per plane ([16 gate rows | 16 up rows] of
+// a gate/up item, 128 rows of a down item) and then a "meta" chunk (the scale
+// rows of the item's matrices and the decode tables of its column blocks; for
+// down items of one column block also the members' h fragments). An item has
+// at most 9 chunks, fewer than the ring's slots, so no copy of an item ever
+// waits for a slot the same item still holds.
 //
 // Consumers: every consumer warp takes every item and multiplies its share of
-// the item's tiles. Partial sums go to a shared-memory slot of the item (one
+// the item's tiles (gate/up: warps 0-7 the gate rows, 8-15 the up rows, each
+// an eighth of the columns). Partial sums go to a shared-memory slot of the item (one
 // slot per queue entry); the warp that finishes last (a shared-memory atomic)
 // reduces them in a fixed order, so results are deterministic, writes
 // h = silu(g) * u (gate/up) or the pair's output rows (down), and moves the
@@ -28,7 +31,7 @@ constexpr int NTHREADS = (NCW + 1) * 32;
 constexpr int NSLOT = 12;                  // ring slots
 constexpr int CHUNK = 16384;               // bytes per ring slot
 constexpr int QDEPTH = 2;                  // item queue (= partial-sum slots): claim at most one item ahead
-constexpr int RED_WORDS = 2 * 16 * 4;      // per warp: [matrix][row][member]
+constexpr int RED_WORDS = 16 * 4;          // per warp: [row][member]
 constexpr int XS_WORDS = (4096 / 32) * 16; // shared copy of the x fragments (T == 1, H <= 4096)
 constexpr int TAB_BYTES = 64;              // decode-table head copied per (block, matrix)
 constexpr uint64_t kDeadlineNs = 200ull * 1000 * 1000;
@@ -40,6 +43,17 @@ struct Desc {
     int c0;   // first chunk of the item
 };
 
+constexpr int UT_MAX = 32; // units (and column blocks) whose layout is staged in shared memory
+
+struct UnitTab {
+    int e, bmax, blk0, nblk;
+    int slot[8]; // slot of each plane of the unit's expert
+};
+
+struct BlkTab {
+    int depth, nmem, pair[4];
+};
+
 struct Smem {
     alignas(128) unsigned char ring[NSLOT][CHUNK];
     float red[QDEPTH][NCW][RED_WORDS];
@@ -49,6 +63,8 @@ struct Smem {
     uint64_t full[NSLOT], empty[NSLOT], qfull[QDEPTH], qempty[QDEPTH];
     Desc q[QDEPTH];
     int cnt[QDEPTH];
+    UnitTab ut[UT_MAX];
+    BlkTab bt[UT_MAX];
 };
 static_assert(sizeof(Smem) <= 227 * 1024, "shared memory of the persistent kernel exceeds one SM's");
 
@@ -60,8 +76,25 @@ struct Args {
     LayerWs W;
 };
 
+// The units' and column blocks' layout: from the shared-memory copy when the
+// call has few of them (decode), else from the workspace.
+struct UnitView {
+    const Smem &S;
+    const LayerWs &W;
+    const int32_t *slot_of;
+    bool staged;
+    __device__ int expert(int u) const { return staged ? S.ut[u].e : __ldg(W.unit_expert + u); }
+    __device__ int bmax(int u) const { return staged ? S.ut[u].bmax : __ldg(W.unit_bmax + u); }
+    __device__ int blk0(int u) const { return staged ? S.ut[u].blk0 : __ldg(W.unit_blk0 + u); }
+    __device__ int nblk(int u) const { return staged ? S.ut[u].nblk : __ldg(W.unit_nblk + u); }
+    __device__ int slot(int u, int e, int p) const { return staged ? S.ut[u].slot[p] : __ldg(slot_of + e * 8 + p); }
+    __device__ int bdepth(int b) const { return staged ? S.bt[b].depth : __ldg(W.blk_depth + b); }
+    __device__ int bnmem(int b) const { return staged ? S.bt[b].nmem : __ldg(W.blk_nmem + b); }
+    __device__ int bpair(int b, int c) const { return staged ? S.bt[b].pair[c] : __ldg(W.blk_pair + b * 4 + c); }
+};
+
 // bytes of an item's meta chunk: scales of its rows, then table heads
-__host__ __device__ inline int meta_bytes_gateup(int H, int G, int nblk) { return 2 * 32 * (H / G) * 4 + nblk * 2 * TAB_BYTES; }
+__host__ __device__ inline int meta_bytes_gateup(int H, int G, int nblk) { return 2 * 16 * (H / G) * 4 + nblk * 2 * TAB_BYTES; }
 __host__ __device__ inline int meta_bytes_down(int I, int G, int nblk) { return 128 * (I / G) * 4 + nblk * TAB_BYTES; }
 // down items with one column block also carry the members' h fragments and exponents
 __host__ __device__ inline int meta_bytes_down_frags(int I, int nmem) { return nmem * (2 * I + hexp_stride(I) * 4); }
@@ -268,21 +301,21 @@ __device__ void h_to_frags(const LayerWs &W, int I, int pair, int Q)
 
 // After the h rows of a gate/up item are written: count the item on its
 // 128-row tile of h; the last one converts the tile and bumps the unit's ready count.
-__device__ void gateup_tile_done(const LayerWs &W, int I, int u, int s32, int blk0, int nblk)
+__device__ void gateup_tile_done(const LayerWs &W, const UnitView &V, int I, int u, int s16, int blk0, int nblk)
 {
     const int lane = threadIdx.x & 31;
     __syncwarp();
     int last = 0;
     if (lane == 0)
-        last = (atom_add_acq_rel(&W.cntH[u * (I / 128) + s32 / 4], 1) == 3);
+        last = (atom_add_acq_rel(&W.cntH[u * (I / 128) + s16 / 8], 1) == 7);
     last = __shfl_sync(0xffffffffu, last, 0);
     __syncwarp();
     if (!last)
         return;
     for (int bi = 0; bi < nblk; ++bi) {
-        const int blk = blk0 + bi, nmem = __ldg(W.blk_nmem + blk);
+        const int blk = blk0 + bi, nmem = V.bnmem(blk);
         for (int c = 0; c < nmem; ++c)
-            h_to_frags(W, I, __ldg(W.blk_pair + blk * 4 + c), s32 / 4);
+            h_to_frags(W, I, V.bpair(blk, c), s16 / 8);
     }
     __syncwarp();
     if (lane == 0)
@@ -360,7 +393,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
     pipe::wait_prerequisites(); // the prep kernel's results are visible from here on
 
     const int nunits = W.flags[kFlagUnits];
-    const int SA = I / 32;  // gate/up items per unit (32 rows of I each)
+    const int SA = I / 16;  // gate/up items per unit (16 rows of I each)
     const int SB = H / 128; // down items per unit (128 rows of H each)
     const int totalA = nunits * SA, total = totalA + nunits * SB;
     const int64_t mat_words = (int64_t)H * I / 32;
@@ -371,6 +404,27 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
             S.xs[i] = W.xfrag[i];
         for (int i = tid; i < H / 128; i += NTHREADS)
             S.xse[i] = W.xexp[i];
+    }
+    // few units (decode): their layout and page-table entries go to shared memory once
+    const int nblocks = W.flags[kFlagBlocks];
+    const UnitView V{S, W, L.slot_of, nunits <= UT_MAX && nblocks <= UT_MAX};
+    if (V.staged) {
+        for (int i = tid; i < nunits * 8; i += NTHREADS) {
+            const int u = i >> 3, p = i & 7, e = __ldg(W.unit_expert + u);
+            S.ut[u].slot[p] = __ldg(L.slot_of + e * 8 + p);
+            if (p == 0) {
+                S.ut[u].e = e;
+                S.ut[u].bmax = __ldg(W.unit_bmax + u);
+                S.ut[u].blk0 = __ldg(W.unit_blk0 + u);
+                S.ut[u].nblk = __ldg(W.unit_nblk + u);
+            }
+        }
+        for (int i = tid; i < nblocks; i += NTHREADS) {
+            S.bt[i].depth = __ldg(W.blk_depth + i);
+            S.bt[i].nmem = __ldg(W.blk_nmem + i);
+            for (int c2 = 0; c2 < 4; ++c2)
+                S.bt[i].pair[c2] = __ldg(W.blk_pair + i * 4 + c2);
+        }
     }
     __syncthreads();
 
@@ -414,30 +468,31 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
             ++qi;
             if (d.kind == 2)
                 break;
-            const int e = __ldg(W.unit_expert + d.u), bmax = __ldg(W.unit_bmax + d.u);
-            const int blk0 = __ldg(W.unit_blk0 + d.u), nblk = __ldg(W.unit_nblk + d.u);
+            const int e = V.expert(d.u), bmax = V.bmax(d.u);
+            const int blk0 = V.blk0(d.u), nblk = V.nblk(d.u);
             const float *esc = L.scales + (int64_t)e * escale_len;
-            // chunk order: gate/up items [gate planes | meta | up planes], down items [planes | meta];
-            // an item's own meta slot is never the one its later chunks wait for (8 < NSLOT).
-            auto issue_planes = [&](int m) {
+            // chunk order [planes | meta]: an item has at most 9 chunks, fewer than NSLOT, so none of
+            // its copies waits for a slot the item itself holds. A gate/up plane chunk holds the
+            // plane's 16 gate rows then its 16 up rows; a down plane chunk 128 rows of the down matrix.
+            auto issue_planes = [&]() {
                 for (int p = 0; p < bmax && ok; ++p) {
                     int s;
                     next_slot(s);
                     if (!ok)
                         break;
-                    const int slot = __ldg(L.slot_of + e * 8 + p);
-                    uint32_t bytes;
-                    int64_t off;
-                    if (d.kind == 0) {
-                        bytes = (uint32_t)(2 * (H / 128) * 256);
-                        off = m * mat_words + (int64_t)d.strip * 2 * (H / 128) * 64;
-                    } else {
-                        bytes = (uint32_t)(8 * (I / 128) * 256);
-                        off = 2 * mat_words + (int64_t)d.strip * 8 * (I / 128) * 64;
-                    }
+                    const int slot = V.slot(d.u, e, p);
+                    const uint32_t bytes = d.kind == 0 ? (uint32_t)(2 * (H / 128) * 256) : (uint32_t)(8 * (I / 128) * 256);
                     if (slot >= 0) {
+                        const uint32_t *base = L.pool + (int64_t)slot * L.slot_words;
                         pipe::mbar_arrive_expect_tx(&S.full[s], bytes);
-                        pipe::bulk_g2s(S.ring[s], L.pool + (int64_t)slot * L.slot_words + off, bytes, &S.full[s]);
+                        if (d.kind == 0) {
+                            const int64_t off = (int64_t)d.strip * (H / 128) * 64;
+                            pipe::bulk_g2s(S.ring[s], base + off, bytes / 2, &S.full[s]);
+                            pipe::bulk_g2s(S.ring[s] + bytes / 2, base + mat_words + off, bytes / 2, &S.full[s]);
+                        } else {
+                            pipe::bulk_g2s(S.ring[s], base + 2 * mat_words + (int64_t)d.strip * 8 * (I / 128) * 64,
+                                           bytes, &S.full[s]);
+                        }
                     } else {
                         // a missing plane: report it and complete the slot without data
                         set_error(W, kErrNoPlane, e * 8 + p);
@@ -452,11 +507,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                 if (!ok)
                     return;
                 if (d.kind == 0) {
-                    const uint32_t sb = 32 * (H / G) * 4;
+                    const uint32_t sb = 16 * (H / G) * 4;
                     pipe::mbar_arrive_expect_tx(&S.full[s], meta_bytes_gateup(H, G, nblk));
                     for (int m = 0; m < 2; ++m)
                         pipe::bulk_g2s(S.ring[s] + m * sb,
-                                       esc + (int64_t)m * I * (H / G) + (int64_t)d.strip * 32 * (H / G), sb, &S.full[s]);
+                                       esc + (int64_t)m * I * (H / G) + (int64_t)d.strip * 16 * (H / G), sb, &S.full[s]);
                     for (int bi = 0; bi < nblk; ++bi)
                         for (int m = 0; m < 2; ++m)
                             pipe::bulk_g2s(S.ring[s] + 2 * sb + (bi * 2 + m) * TAB_BYTES,
@@ -466,7 +521,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                     int nmem = 0;
                     if (nblk == 1) {
                         // the h fragments come along: wait (bounded) until the unit's h is converted
-                        nmem = __ldg(W.blk_nmem + blk0);
+                        nmem = V.bnmem(blk0);
                         while (pipe::ld_acquire(&W.readyB[d.u]) < I / 128) {
                             if (pipe::globaltimer() > deadline) {
                                 set_error(W, kErrTimeout, 5);
@@ -484,7 +539,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                                        W.tabs + ((int64_t)(blk0 + bi) * 3 + 2) * kTabWords, TAB_BYTES, &S.full[s]);
                     unsigned char *fb = S.ring[s] + sb + nblk * TAB_BYTES;
                     for (int c2 = 0; c2 < nmem; ++c2) {
-                        const int pair = __ldg(W.blk_pair + blk0 * 4 + c2);
+                        const int pair = V.bpair(blk0, c2);
                         pipe::bulk_g2s(fb + c2 * 2 * I, W.hfrag + (int64_t)pair * (I / 32) * 16, 2 * I, &S.full[s]);
                         pipe::bulk_g2s(fb + nmem * 2 * I + c2 * hexp_stride(I) * 4,
                                        W.hexp + (int64_t)pair * hexp_stride(I), hexp_stride(I) * 4, &S.full[s]);
@@ -492,17 +547,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                 }
                 ++c;
             };
-            if (d.kind == 0) {
-                issue_planes(0);
-                if (ok)
-                    issue_meta();
-                if (ok)
-                    issue_planes(1);
-            } else {
-                issue_planes(0);
-                if (ok)
-                    issue_meta();
-            }
+            issue_planes();
+            if (ok)
+                issue_meta();
         }
         // no copy may still be landing in shared memory when the CTA exits
         for (int cc = (c > NSLOT ? c - NSLOT : 0); cc < c; ++cc)
@@ -521,43 +568,44 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
         const Desc d = S.q[qs];
         if (d.kind == 2)
             break;
-        const int blk0 = __ldg(W.unit_blk0 + d.u);
-        const int nblk = __ldg(W.unit_nblk + d.u), bmax = __ldg(W.unit_bmax + d.u);
+        const int blk0 = V.blk0(d.u);
+        const int nblk = V.nblk(d.u), bmax = V.bmax(d.u);
         const bool fast = (nblk == 1);
         float *red = S.red[qs][warp];
         bool fine = true;
-        const int cm = d.c0 + bmax; // meta chunk (after the first matrix's planes)
+        const int cm = d.c0 + bmax; // meta chunk (after the item's planes)
         const unsigned char *meta = S.ring[cm % NSLOT];
         if (!pipe::mbar_wait(&S.full[cm % NSLOT], (cm / NSLOT) & 1, deadline))
             fine = false;
 
         if (d.kind == 0) {
-            // gate/up: warp -> strip sr (of 2 x 16 rows) and K part kp (of 8)
-            const int sr = warp >> 3, kp = warp & 7, tpw = (H / 128) / 8, Q0 = kp * tpw;
-            const int tix0 = sr * (H / 128) + Q0;
+            // gate/up: warp -> matrix m (warps 0-7 gate, 8-15 up) and K part kp (of 8) of the
+            // item's 16 rows; a plane chunk holds [gate rows | up rows] of one plane
+            const int m = warp >> 3, kp = warp & 7, tpw = (H / 128) / 8, Q0 = kp * tpw;
+            const int tix0 = m * (H / 128) + Q0;
             const int ngr = H / G;
-            for (int m = 0; m < 2; ++m) {
-                const unsigned char *pp[8];
+            const unsigned char *pp[8];
 #pragma unroll
-                for (int p = 0; p < 8; ++p) {
-                    const int cc = d.c0 + m * (bmax + 1) + p;
-                    pp[p] = S.ring[cc % NSLOT] + tix0 * 256 + lane * 8;
-                    if (p < bmax && !pipe::mbar_wait(&S.full[cc % NSLOT], (cc / NSLOT) & 1, deadline))
-                        fine = false;
-                }
-                const float *sc0 = reinterpret_cast<const float *>(meta) + (m * 32 + 16 * sr + g) * ngr + Q0 * (128 / G);
+            for (int p = 0; p < 8; ++p) {
+                const int cc = d.c0 + p;
+                pp[p] = S.ring[cc % NSLOT] + tix0 * 256 + lane * 8;
+                if (p < bmax && !pipe::mbar_wait(&S.full[cc % NSLOT], (cc / NSLOT) & 1, deadline))
+                    fine = false;
+            }
+            {
+                const float *sc0 = reinterpret_cast<const float *>(meta) + (m * 16 + g) * ngr + Q0 * (128 / G);
                 const float *sc1 = sc0 + 8 * ngr;
                 for (int bi = 0; bi < nblk; ++bi) {
                     const int blk = blk0 + bi;
-                    const int dd = __ldg(W.blk_depth + blk), nmem = __ldg(W.blk_nmem + blk);
+                    const int dd = V.bdepth(blk), nmem = V.bnmem(blk);
                     const int c = g >> 1;
                     float acc0 = 0.0f, acc1 = 0.0f;
                     const int *exps = nullptr;
                     if (t < nmem) {
-                        const int tok = __ldg(W.blk_pair + blk * 4 + t) / k;
+                        const int tok = V.bpair(blk, t) / k;
                         exps = stage_x ? S.xse : W.xexp + (int64_t)tok * (H / 128);
                     }
-                    const unsigned char *tabs = meta + 2 * 32 * ngr * 4 + (bi * 2 + m) * TAB_BYTES;
+                    const unsigned char *tabs = meta + 2 * 16 * ngr * 4 + (bi * 2 + m) * TAB_BYTES;
                     const uint32_t *big = W.tabs + ((int64_t)blk * 3 + m) * kTabWords + 16;
                     if (stage_x) {
                         const bool has = c < nmem;
@@ -567,28 +615,28 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                     } else {
                         const uint32_t *fptr = nullptr;
                         if (c < nmem) {
-                            const int tok = __ldg(W.blk_pair + blk * 4 + c) / k;
+                            const int tok = V.bpair(blk, c) / k;
                             fptr = W.xfrag + (int64_t)tok * (H / 32) * 16 + Q0 * 64 + (4 * (g & 1) + t) * 2;
                         }
                         warp_block_any<GS, 1>(dd, pp, tpw, Q0, tabs, big, fptr, 16, exps, sc0, sc1, acc0, acc1);
                     }
                     if (t < nmem) {
                         if (fast) {
-                            red[(m * 16 + g) * 4 + t] = acc0;
-                            red[(m * 16 + g + 8) * 4 + t] = acc1;
+                            red[g * 4 + t] = acc0;
+                            red[(g + 8) * 4 + t] = acc1;
                         } else {
-                            const int pair = __ldg(W.blk_pair + blk * 4 + t);
-                            float *dst = W.pA + (((int64_t)pair * (I / 16) + 2 * d.strip + sr) * 8 + kp) * 32 + m * 16;
+                            const int pair = V.bpair(blk, t);
+                            float *dst = W.pA + (((int64_t)pair * (I / 16) + d.strip) * 8 + kp) * 32 + m * 16;
                             __stcg(dst + g, acc0);
                             __stcg(dst + g + 8, acc1);
                         }
                     }
                 }
-                __syncwarp();
-                if (lane == 0)
-                    for (int p = 0; p < bmax; ++p)
-                        pipe::mbar_arrive(&S.empty[(d.c0 + m * (bmax + 1) + p) % NSLOT]);
             }
+            __syncwarp();
+            if (lane == 0)
+                for (int p = 0; p < bmax; ++p)
+                    pipe::mbar_arrive(&S.empty[(d.c0 + p) % NSLOT]);
             __syncwarp();
             if (lane == 0)
                 pipe::mbar_arrive(&S.empty[cm % NSLOT]);
@@ -604,35 +652,36 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
             last = __shfl_sync(0xffffffffu, last, 0);
             __syncwarp();
             if (last) {
-                // h rows of the item: lane = row (32 rows), every member of every block
+                // h rows of the item: lanes 0-15 = row, every member of every block
                 if (fast)
                     __threadfence_block();
                 for (int bi = 0; bi < nblk; ++bi) {
-                    const int blk = blk0 + bi, nmem = __ldg(W.blk_nmem + blk);
+                    const int blk = blk0 + bi, nmem = V.bnmem(blk);
                     for (int c = 0; c < nmem; ++c) {
-                        const int pair = __ldg(W.blk_pair + blk * 4 + c);
-                        const int s16 = lane >> 4, rr = lane & 15;
+                        const int pair = V.bpair(blk, c);
+                        const int rr = lane & 15;
                         float gv = 0.0f, uv = 0.0f;
                         if (fast) {
 #pragma unroll
                             for (int kq = 0; kq < 8; ++kq) {
-                                gv += S.red[qs][8 * s16 + kq][(0 * 16 + rr) * 4 + c];
-                                uv += S.red[qs][8 * s16 + kq][(1 * 16 + rr) * 4 + c];
+                                gv += S.red[qs][kq][rr * 4 + c];
+                                uv += S.red[qs][8 + kq][rr * 4 + c];
                             }
                         } else {
-                            const float *src = W.pA + (((int64_t)pair * (I / 16) + 2 * d.strip + s16) * 8) * 32;
+                            const float *src = W.pA + (((int64_t)pair * (I / 16) + d.strip) * 8) * 32;
 #pragma unroll
                             for (int kq = 0; kq < 8; ++kq) {
                                 gv += __ldcg(src + kq * 32 + rr);
                                 uv += __ldcg(src + kq * 32 + 16 + rr);
                             }
                         }
-                        __stcg(W.h + (int64_t)pair * I + 32 * d.strip + lane, gv / (1.0f + expf(-gv)) * uv);
+                        if (lane < 16)
+                            __stcg(W.h + (int64_t)pair * I + 16 * d.strip + rr, gv / (1.0f + expf(-gv)) * uv);
                     }
                 }
                 if (fast && lane == 0)
                     S.cnt[qs] = 0;
-                gateup_tile_done(W, I, d.u, d.strip, blk0, nblk);
+                gateup_tile_done(W, V, I, d.u, d.strip, blk0, nblk);
             }
         } else {
             // down: warp -> strip sb (of 8 x 16 rows) and K part kp (of 2)
@@ -662,7 +711,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
             const float *sc1 = sc0 + 8 * ngr;
             for (int bi = 0; bi < nblk; ++bi) {
                 const int blk = blk0 + bi;
-                const int dd = __ldg(W.blk_depth + blk), nmem = __ldg(W.blk_nmem + blk);
+                const int dd = V.bdepth(blk), nmem = V.bnmem(blk);
                 const int c = g >> 1;
                 float acc0 = 0.0f, acc1 = 0.0f;
                 const unsigned char *tabs = meta + 128 * ngr * 4 + bi * TAB_BYTES;
@@ -679,12 +728,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                 } else {
                     const uint32_t *fptr = nullptr;
                     if (c < nmem) {
-                        const int pair = __ldg(W.blk_pair + blk * 4 + c);
+                        const int pair = V.bpair(blk, c);
                         fptr = W.hfrag + (int64_t)pair * (I / 32) * 16 + Q0 * 64 + (4 * (g & 1) + t) * 2;
                     }
                     const int *exps = nullptr;
                     if (t < nmem)
-                        exps = W.hexp + (int64_t)__ldg(W.blk_pair + blk * 4 + t) * hexp_stride(I);
+                        exps = W.hexp + (int64_t)V.bpair(blk, t) * hexp_stride(I);
                     warp_block_any<GS, 2>(dd, pp, tpw, Q0, tabs, big, fptr, 16, exps, sc0, sc1, acc0, acc1);
                 }
                 if (t < nmem) {
@@ -692,7 +741,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                         red[g * 4 + t] = acc0;
                         red[(g + 8) * 4 + t] = acc1;
                     } else {
-                        const int pair = __ldg(W.blk_pair + blk * 4 + t);
+                        const int pair = V.bpair(blk, t);
                         float *dst = W.pB + (((int64_t)pair * (H / 16) + 8 * d.strip + sb) * 2 + kp) * 16;
                         __stcg(dst + g, acc0);
                         __stcg(dst + g + 8, acc1);
@@ -720,9 +769,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                 if (fast)
                     __threadfence_block();
                 for (int bi = 0; bi < nblk; ++bi) {
-                    const int blk = blk0 + bi, nmem = __ldg(W.blk_nmem + blk);
+                    const int blk = blk0 + bi, nmem = V.bnmem(blk);
                     for (int c = 0; c < nmem; ++c) {
-                        const int pair = __ldg(W.blk_pair + blk * 4 + c);
+                        const int pair = V.bpair(blk, c);
                         for (int r = lane; r < 128; r += 32) {
                             const int s8 = r >> 4, rr = r & 15;
                             float v;
@@ -739,9 +788,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                 if (fast && lane == 0)
                     S.cnt[qs] = 0;
                 for (int bi = 0; bi < nblk; ++bi) {
-                    const int blk = blk0 + bi, nmem = __ldg(W.blk_nmem + blk);
+                    const int blk = blk0 + bi, nmem = V.bnmem(blk);
                     for (int c = 0; c < nmem; ++c)
-                        down_rows_done(a, __ldg(W.blk_pair + blk * 4 + c), d.strip);
+                        down_rows_done(a, V.bpair(blk, c), d.strip);
                 }
             }
         }
