@@ -27,7 +27,7 @@
 namespace mk {
 
 constexpr int NCW = 16;                    // consumer warps
-constexpr int NTHREADS = (NCW + 1) * 32;
+constexpr int NTHREADS = (NCW + 2) * 32; // + producer warp + epilogue warp
 constexpr int NSLOT = 12;                  // ring slots
 constexpr int CHUNK = 16384;               // bytes per ring slot
 constexpr int QDEPTH = 2;                  // item queue (= partial-sum slots): claim at most one item ahead
@@ -60,7 +60,7 @@ struct Smem {
     uint32_t xs[XS_WORDS];
     uint32_t zeros[4];
     int xse[32];
-    uint64_t full[NSLOT], empty[NSLOT], qfull[QDEPTH], qempty[QDEPTH];
+    uint64_t full[NSLOT], empty[NSLOT], qfull[QDEPTH], qempty[QDEPTH], epi[QDEPTH];
     Desc q[QDEPTH];
     int cnt[QDEPTH];
     UnitTab ut[UT_MAX];
@@ -382,7 +382,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
         }
         for (int s = 0; s < QDEPTH; ++s) {
             pipe::mbar_init(&S.qfull[s], 1);
-            pipe::mbar_init(&S.qempty[s], NCW);
+            pipe::mbar_init(&S.qempty[s], NCW + 1); // consumers + epilogue warp
+            pipe::mbar_init(&S.epi[s], 1);
             S.cnt[s] = 0;
         }
         pipe::fence_barrier_init();
@@ -557,6 +558,88 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
         return;
     }
 
+    if (warp == NCW + 1) {
+        // ------------------------------------------------------------ epilogue warp
+        // Items of one column block: once the last consumer warp has handed the item over,
+        // reduce its shared-memory partials in a fixed order, release the queue slot, then do
+        // the item's global work (h rows and the tile count, or the pair's output rows and the
+        // slot-order combine) while the consumers already work on the next items.
+        uint32_t epi_phase = 0; // bit qs: parity of the next phase of epi[qs] (only handed-over items use it)
+        for (int qi = 0;; ++qi) {
+            const int qs = qi % QDEPTH;
+            if (!pipe::mbar_wait(&S.qfull[qs], (qi / QDEPTH) & 1, deadline)) {
+                set_error(W, kErrTimeout, 7);
+                break;
+            }
+            const Desc d = S.q[qs];
+            if (d.kind == 2)
+                break;
+            const int blk0 = V.blk0(d.u);
+            if (V.nblk(d.u) != 1) {
+                // several column blocks: the consumers' last warp does it through global memory
+                __syncwarp();
+                if (lane == 0)
+                    pipe::mbar_arrive(&S.qempty[qs]);
+                continue;
+            }
+            if (!pipe::mbar_wait(&S.epi[qs], (epi_phase >> qs) & 1u, deadline)) {
+                set_error(W, kErrTimeout, 8);
+                break;
+            }
+            epi_phase ^= 1u << qs;
+            const int nmem = V.bnmem(blk0);
+            if (d.kind == 0) {
+                // h rows: lanes 0-15 = row, one value per member
+                const int rr = lane & 15;
+                float hv[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float gv = 0.0f, uv = 0.0f;
+                    if (c < nmem) {
+#pragma unroll
+                        for (int kq = 0; kq < 8; ++kq) {
+                            gv += S.red[qs][kq][rr * 4 + c];
+                            uv += S.red[qs][8 + kq][rr * 4 + c];
+                        }
+                    }
+                    hv[c] = gv / (1.0f + expf(-gv)) * uv;
+                }
+                __syncwarp();
+                if (lane == 0)
+                    pipe::mbar_arrive(&S.qempty[qs]);
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    if (c < nmem && lane < 16)
+                        __stcg(W.h + (int64_t)V.bpair(blk0, c) * I + 16 * d.strip + rr, hv[c]);
+                gateup_tile_done(W, V, I, d.u, d.strip, blk0, 1);
+            } else {
+                // output rows: lane owns rows lane + 32*i
+                float ov[4][4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int r = lane + 32 * i, s8 = r >> 4, rr = r & 15;
+                        ov[c][i] = c < nmem ? S.red[qs][2 * s8][rr * 4 + c] + S.red[qs][2 * s8 + 1][rr * 4 + c] : 0.0f;
+                    }
+                __syncwarp();
+                if (lane == 0)
+                    pipe::mbar_arrive(&S.qempty[qs]);
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    if (c < nmem) {
+                        const int pair = V.bpair(blk0, c);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            __stcg(W.part + (int64_t)pair * H + 128 * d.strip + lane + 32 * i, ov[c][i]);
+                    }
+                for (int c = 0; c < nmem; ++c)
+                    down_rows_done(a, V.bpair(blk0, c), d.strip);
+            }
+        }
+        return;
+    }
+
     // ---------------------------------------------------------------- consumers
     const int g = lane >> 2, t = lane & 3;
     for (int qi = 0;; ++qi) {
@@ -642,9 +725,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                 pipe::mbar_arrive(&S.empty[cm % NSLOT]);
             int last = 0;
             if (fast) {
+                // the epilogue warp reduces the partials; the last warp only hands the item over
                 if (lane == 0) {
                     __threadfence_block();
-                    last = (atomicAdd(&S.cnt[qs], 1) == NCW - 1);
+                    if (atomicAdd(&S.cnt[qs], 1) == NCW - 1) {
+                        S.cnt[qs] = 0;
+                        pipe::mbar_arrive(&S.epi[qs]);
+                    }
                 }
             } else if (lane == 0) {
                 last = (atom_add_acq_rel(&W.cntA[d.u * SA + d.strip], 1) == NCW - 1);
@@ -653,34 +740,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
             __syncwarp();
             if (last) {
                 // h rows of the item: lanes 0-15 = row, every member of every block
-                if (fast)
-                    __threadfence_block();
                 for (int bi = 0; bi < nblk; ++bi) {
                     const int blk = blk0 + bi, nmem = V.bnmem(blk);
                     for (int c = 0; c < nmem; ++c) {
                         const int pair = V.bpair(blk, c);
                         const int rr = lane & 15;
                         float gv = 0.0f, uv = 0.0f;
-                        if (fast) {
+                        const float *src = W.pA + (((int64_t)pair * (I / 16) + d.strip) * 8) * 32;
 #pragma unroll
-                            for (int kq = 0; kq < 8; ++kq) {
-                                gv += S.red[qs][kq][rr * 4 + c];
-                                uv += S.red[qs][8 + kq][rr * 4 + c];
-                            }
-                        } else {
-                            const float *src = W.pA + (((int64_t)pair * (I / 16) + d.strip) * 8) * 32;
-#pragma unroll
-                            for (int kq = 0; kq < 8; ++kq) {
-                                gv += __ldcg(src + kq * 32 + rr);
-                                uv += __ldcg(src + kq * 32 + 16 + rr);
-                            }
+                        for (int kq = 0; kq < 8; ++kq) {
+                            gv += __ldcg(src + kq * 32 + rr);
+                            uv += __ldcg(src + kq * 32 + 16 + rr);
                         }
                         if (lane < 16)
                             __stcg(W.h + (int64_t)pair * I + 16 * d.strip + rr, gv / (1.0f + expf(-gv)) * uv);
                     }
                 }
-                if (fast && lane == 0)
-                    S.cnt[qs] = 0;
                 gateup_tile_done(W, V, I, d.u, d.strip, blk0, nblk);
             }
         } else {
@@ -758,7 +833,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
             if (fast) {
                 if (lane == 0) {
                     __threadfence_block();
-                    last = (atomicAdd(&S.cnt[qs], 1) == NCW - 1);
+                    if (atomicAdd(&S.cnt[qs], 1) == NCW - 1) {
+                        S.cnt[qs] = 0;
+                        pipe::mbar_arrive(&S.epi[qs]);
+                    }
                 }
             } else if (lane == 0) {
                 last = (atom_add_acq_rel(&W.cntB[d.u * SB + d.strip], 1) == NCW - 1);
@@ -766,27 +844,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
             last = __shfl_sync(0xffffffffu, last, 0);
             __syncwarp();
             if (last) {
-                if (fast)
-                    __threadfence_block();
                 for (int bi = 0; bi < nblk; ++bi) {
                     const int blk = blk0 + bi, nmem = V.bnmem(blk);
                     for (int c = 0; c < nmem; ++c) {
                         const int pair = V.bpair(blk, c);
                         for (int r = lane; r < 128; r += 32) {
                             const int s8 = r >> 4, rr = r & 15;
-                            float v;
-                            if (fast) {
-                                v = S.red[qs][2 * s8][rr * 4 + c] + S.red[qs][2 * s8 + 1][rr * 4 + c];
-                            } else {
-                                const float *src = W.pB + (((int64_t)pair * (H / 16) + 8 * d.strip + s8) * 2) * 16;
-                                v = __ldcg(src + rr) + __ldcg(src + 16 + rr);
-                            }
-                            __stcg(W.part + (int64_t)pair * H + 128 * d.strip + r, v);
+                            const float *src = W.pB + (((int64_t)pair * (H / 16) + 8 * d.strip + s8) * 2) * 16;
+                            __stcg(W.part + (int64_t)pair * H + 128 * d.strip + r, __ldcg(src + rr) + __ldcg(src + 16 + rr));
                         }
                     }
                 }
-                if (fast && lane == 0)
-                    S.cnt[qs] = 0;
                 for (int bi = 0; bi < nblk; ++bi) {
                     const int blk = blk0 + bi, nmem = V.bnmem(blk);
                     for (int c = 0; c < nmem; ++c)
