@@ -112,7 +112,7 @@ struct PrepArgs {
     LayerWs W;
 };
 
-constexpr int kPrepThreads = 512;
+constexpr int kPrepThreads = 1024;
 
 __global__ void __launch_bounds__(kPrepThreads) layer_prep_kernel(PrepArgs a)
 {
@@ -142,7 +142,10 @@ __global__ void __launch_bounds__(kPrepThreads) layer_prep_kernel(PrepArgs a)
         for (int tok = warp; tok < T; tok += n_rw) {
             int id;
             float wt;
-            dev::route_token(a.logits + (int64_t)tok * E, E, k, stage, id, wt);
+            if (E <= 512)
+                dev::route_token_reg<16>(a.logits + (int64_t)tok * E, E, k, id, wt);
+            else
+                dev::route_token(a.logits + (int64_t)tok * E, E, k, stage, id, wt);
             const float v = (lane < k) ? __fmul_rn(wt, __ldg(a.sens + id)) : 0.0f;
             const int b = dev::select_token(v, k, a.B, nullptr);
             if (lane < k) {

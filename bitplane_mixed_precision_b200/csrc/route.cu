@@ -55,7 +55,10 @@ __global__ void route_kernel(const float *__restrict__ logits, int T, int E, int
         return;
     int id;
     float wt;
-    dev::route_token(logits + (int64_t)warp * E, E, k, stage, id, wt);
+    if (E <= 512)
+        dev::route_token_reg<16>(logits + (int64_t)warp * E, E, k, id, wt);
+    else
+        dev::route_token(logits + (int64_t)warp * E, E, k, stage, id, wt);
     const int lane = threadIdx.x & 31;
     if (lane < k) {
         ids[warp * k + lane] = id;

@@ -65,6 +65,55 @@ __device__ __forceinline__ void route_token(const float *__restrict__ l, int E, 
     w_out = (lane < k) ? __double2float_rn(__ddiv_rn(e, sum)) : 0.0f;
 }
 
+// route_token for E <= 32*NPL with the logits' keys in registers (NPL per lane,
+// every index compile-time): the same picks, ties and weights.
+template <int NPL>
+__device__ __forceinline__ void route_token_reg(const float *__restrict__ l, int E, int k, int &id_out, float &w_out)
+{
+    const int lane = threadIdx.x & 31;
+    uint32_t key[NPL];
+#pragma unroll
+    for (int j = 0; j < NPL; ++j)
+        key[j] = (lane + 32 * j < E) ? ord_key(__ldg(l + lane + 32 * j)) : 0u;
+    uint32_t bk;
+    int bj;
+    auto local_best = [&]() {
+        bk = 0u;
+        bj = -1;
+#pragma unroll
+        for (int j = 0; j < NPL; ++j)
+            if (key[j] > bk) {
+                bk = key[j];
+                bj = j;
+            }
+    };
+    local_best();
+    int my_id = 0;
+    for (int s = 0; s < k; ++s) {
+        const uint32_t gmax = __reduce_max_sync(0xffffffffu, bk);
+        const unsigned cand = (bj >= 0 && bk == gmax) ? (unsigned)(lane + 32 * bj) : 0x7fffffffu;
+        const unsigned win = __reduce_min_sync(0xffffffffu, cand);
+        if (lane == s)
+            my_id = (int)win;
+        if (lane == (int)(win & 31u)) {
+            const int jw = (int)(win >> 5);
+#pragma unroll
+            for (int j = 0; j < NPL; ++j)
+                if (j == jw)
+                    key[j] = 0u;
+            local_best();
+        }
+    }
+    const float my_l = (lane < k) ? __ldg(l + my_id) : 0.0f;
+    const double l0 = (double)__shfl_sync(0xffffffffu, my_l, 0);
+    const double e = (lane < k) ? exp((double)my_l - l0) : 0.0;
+    double sum = 0.0;
+    for (int s = 0; s < k; ++s)
+        sum = __dadd_rn(sum, __shfl_sync(0xffffffffu, e, s));
+    id_out = my_id;
+    w_out = (lane < k) ? __double2float_rn(__ddiv_rn(e, sum)) : 0.0f;
+}
+
 // Greedy prefix selection for one token (transcript cue 29): lane i < k holds
 // v_i = w_i * s_{e_i}; B - k rounds grant one bit to the largest v_i * 2^-b_i
 // (exact ldexp; ties to the lower slot; 8-bit slots skipped). Returns b_i.
