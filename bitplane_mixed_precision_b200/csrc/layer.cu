@@ -47,6 +47,7 @@ LayerWs carve_layer_ws(void *ws, int T, int k, int H, int I, size_t *bytes)
     const size_t o_flags = take(64 * 4);
     const size_t o_bd = take(P * 4), o_bn = take(P * 4), o_bp = take(P * 16), o_be = take(P * 4);
     const size_t o_ue = take(P * 4), o_u0 = take(P * 4), o_un = take(P * 4), o_ub = take(P * 4);
+    const size_t o_ut = take(P * 12 * 4);
     const size_t o_ca = take(P * (I / 16) * 4), o_ch = take(P * (I / 128) * 4), o_rb = take(P * 4);
     const size_t o_cb = take(P * (H / 128) * 4), o_yc = take((size_t)T * (H / 128) * 4);
     const size_t o_pa = take(P * (size_t)(I / 16) * 8 * 32 * 4), o_pb = take(P * (size_t)(H / 16) * 2 * 16 * 4);
@@ -71,6 +72,7 @@ LayerWs carve_layer_ws(void *ws, int T, int k, int H, int I, size_t *bytes)
     L.unit_blk0 = reinterpret_cast<int *>(b + o_u0);
     L.unit_nblk = reinterpret_cast<int *>(b + o_un);
     L.unit_bmax = reinterpret_cast<int *>(b + o_ub);
+    L.utab = reinterpret_cast<int *>(b + o_ut);
     L.cntA = reinterpret_cast<int *>(b + o_ca);
     L.cntH = reinterpret_cast<int *>(b + o_ch);
     L.readyB = reinterpret_cast<int *>(b + o_rb);
@@ -240,6 +242,14 @@ __global__ void __launch_bounds__(kPrepThreads) layer_prep_kernel(PrepArgs a)
         W.unit_blk0[rank] = u_b0[i];
         W.unit_nblk[rank] = u_nb[i];
         W.unit_bmax[rank] = u_bm[i];
+        // the same unit as one record with its page-table entries, for the persistent kernel
+        int *ut = W.utab + rank * 12;
+        ut[0] = u_e[i];
+        ut[1] = u_bm[i];
+        ut[2] = u_b0[i];
+        ut[3] = u_nb[i];
+        for (int p = 0; p < 8; ++p)
+            ut[4 + p] = __ldg(a.L.slot_of + u_e[i] * 8 + p);
     }
     // 4. decode tables: one warp per (block, matrix)
     for (int j = warp; j < nb * 3; j += nwarps) {

@@ -32,6 +32,7 @@ struct LayerWs {
     int *blk_pair;   //   [4] pair index t*k + i of each member
     int *blk_expert; //   expert
     int *unit_expert, *unit_blk0, *unit_nblk, *unit_bmax; // per unit (one expert, <= 4 blocks)
+    int *utab;       // per unit, 12 ints: expert, bmax, blk0, nblk, slot of planes 0..7
     int *cntA;       // per gate/up item (unit, 16 rows of I): consumer warps finished
     int *cntH;       // per (unit, 128 rows of I): gate/up items finished (8 per tile)
     int *readyB;     // per unit: 128-row tiles of h turned into fragments

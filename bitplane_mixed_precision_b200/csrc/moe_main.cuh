@@ -410,16 +410,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
     const int nblocks = W.flags[kFlagBlocks];
     const UnitView V{S, W, L.slot_of, nunits <= UT_MAX && nblocks <= UT_MAX};
     if (V.staged) {
-        for (int i = tid; i < nunits * 8; i += NTHREADS) {
-            const int u = i >> 3, p = i & 7, e = __ldg(W.unit_expert + u);
-            S.ut[u].slot[p] = __ldg(L.slot_of + e * 8 + p);
-            if (p == 0) {
-                S.ut[u].e = e;
-                S.ut[u].bmax = __ldg(W.unit_bmax + u);
-                S.ut[u].blk0 = __ldg(W.unit_blk0 + u);
-                S.ut[u].nblk = __ldg(W.unit_nblk + u);
-            }
-        }
+        static_assert(sizeof(UnitTab) == 12 * sizeof(int), "unit record layout");
+        for (int i = tid; i < nunits * 12; i += NTHREADS)
+            reinterpret_cast<int *>(S.ut)[i] = __ldg(W.utab + i);
         for (int i = tid; i < nblocks; i += NTHREADS) {
             S.bt[i].depth = __ldg(W.blk_depth + i);
             S.bt[i].nmem = __ldg(W.blk_nmem + i);
@@ -450,7 +443,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                 break;
             }
             Desc d;
-            const int u = atomicAdd(&W.flags[kFlagSched], 1);
+            // the first item of each SM is its own index; the counter hands out the rest
+            const int u = (qi == 0) ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(&W.flags[kFlagSched], 1);
             if (u >= total) {
                 d.kind = 2;
                 d.u = d.strip = 0;
