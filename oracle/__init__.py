@@ -55,6 +55,7 @@ def _l():
                               i32], i32),
             "or_cache_sim_prefix": ([i32, i32, i64, i64, P, P, P, P, P, P, i64, P, P], i32),
             "or_cache_sim_independent": ([i32, i32, i64, i64, P, P, P, P, P, P], i32),
+            "or_cache_sim_independent_down": ([i32, i32, i64, i64, P, P, P, P, P, P], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -239,4 +240,20 @@ def cache_sim_independent(L: int, E: int, cap_planes: int, layer, expert, depth,
                                        _p(batch), _p(hit), ctypes.byref(fetched))
     if rc:
         raise ValueError(f"or_cache_sim_independent failed ({rc})")
+    return hit, fetched.value
+
+
+def cache_sim_independent_down(L: int, E: int, cap_planes: int, layer, expert, depth, batch):
+    """Independent objects with downward reuse: (hit uint8 [n], planes fetched)."""
+    layer = np.ascontiguousarray(layer, dtype=np.int32)
+    expert = np.ascontiguousarray(expert, dtype=np.int32)
+    depth = np.ascontiguousarray(depth, dtype=np.uint8)
+    batch = np.ascontiguousarray(batch, dtype=np.int32)
+    n = len(layer)
+    hit = np.empty(n, dtype=np.uint8)
+    fetched = ctypes.c_int64(0)
+    rc = _l().or_cache_sim_independent_down(L, E, cap_planes, n, _p(layer), _p(expert), _p(depth),
+                                            _p(batch), _p(hit), ctypes.byref(fetched))
+    if rc:
+        raise ValueError(f"or_cache_sim_independent_down failed ({rc})")
     return hit, fetched.value

@@ -592,3 +592,70 @@ int or_cache_sim_independent(int L, int E, int64_t cap_planes, int64_t n_acc,
     free(list);
     return rc;
 }
+
+/*
+ * Independent objects with downward reuse [T#51]: one resident copy per
+ * (layer, expert) at some depth r (r planes, loaded as one object). An access
+ * at depth b hits when r >= b (the deeper copy serves the shallower request);
+ * otherwise the copy is promoted: a whole new object of b planes is fetched
+ * (objects share no bits) and replaces the old one. Whole objects are evicted
+ * least-recently-used first (not those accessed in the current batch) until
+ * the new one fits in the same plane capacity.
+ * Outputs per access: 1 on hit, 0 on miss; *planes_fetched.
+ */
+int or_cache_sim_independent_down(int L, int E, int64_t cap_planes, int64_t n_acc,
+                                  const int32_t *acc_layer, const int32_t *acc_expert,
+                                  const uint8_t *acc_depth, const int32_t *acc_batch,
+                                  uint8_t *hit, int64_t *planes_fetched)
+{
+    int64_t NE = (int64_t)L * E;
+    uint8_t *dep = (uint8_t *)calloc((size_t)NE, 1);
+    int64_t *ts = (int64_t *)malloc(sizeof(int64_t) * (size_t)NE);
+    int32_t *last_batch = (int32_t *)malloc(sizeof(int32_t) * (size_t)NE);
+    if (!dep || !ts || !last_batch)
+        return 2;
+    int64_t used = 0, fetched = 0;
+    int rc = 0;
+    for (int64_t a = 0; a < n_acc; ++a) {
+        int l = acc_layer[a], e = acc_expert[a], b = acc_depth[a];
+        if (l < 0 || l >= L || e < 0 || e >= E || b < 1 || b > 8) {
+            rc = 1;
+            break;
+        }
+        int64_t x = (int64_t)l * E + e;
+        last_batch[x] = acc_batch[a];
+        ts[x] = a;
+        if (dep[x] >= b) {
+            hit[a] = 1;
+            continue;
+        }
+        hit[a] = 0;
+        used -= dep[x]; /* the old copy is replaced */
+        dep[x] = 0;
+        while (used + b > cap_planes) {
+            int64_t victim = -1;
+            for (int64_t y = 0; y < NE; ++y) {
+                if (dep[y] == 0 || last_batch[y] == acc_batch[a])
+                    continue;
+                if (victim < 0 || ts[y] < ts[victim])
+                    victim = y;
+            }
+            if (victim < 0) {
+                rc = 3;
+                break;
+            }
+            used -= dep[victim];
+            dep[victim] = 0;
+        }
+        if (rc)
+            break;
+        dep[x] = (uint8_t)b;
+        used += b;
+        fetched += b;
+    }
+    *planes_fetched = fetched;
+    free(dep);
+    free(ts);
+    free(last_batch);
+    return rc;
+}

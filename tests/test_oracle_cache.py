@@ -86,3 +86,60 @@ def test_independent_objects_hit_only_exact_precision(oracle_mod):
     # the prefix cache serves the same trace with 4 planes fetched in total
     _, _, fp = oracle_mod.cache_sim_prefix(1, 4, 64, acc[:, 0], acc[:, 1], acc[:, 2], acc[:, 3])
     assert fp == 4
+
+
+# Independent objects with downward reuse (transcript cue 51: a resident higher-precision copy
+# serves lower-bit requests and is promoted when a request needs more).
+
+def _down(oracle_mod, cap, accesses, L=1, E=8):
+    a = np.array(accesses, dtype=np.int64)
+    return oracle_mod.cache_sim_independent_down(L, E, cap, a[:, 0], a[:, 1], a[:, 2], a[:, 3])
+
+
+def test_downward_reuse_hand_traces(oracle_mod):
+    # 6 resident, 3 requested: served by the deeper copy (an exact-object cache misses here)
+    hit, fetched = _down(oracle_mod, 64, [(0, 1, 6, 0), (0, 1, 3, 1)])
+    assert list(hit) == [0, 1] and fetched == 6
+    hit_i, fetched_i = oracle_mod.cache_sim_independent(1, 8, 64, [0, 0], [1, 1], [6, 3], [0, 1])
+    assert list(hit_i) == [0, 0] and fetched_i == 9
+    # 3 resident, 5 requested: promoted by loading a whole 5-plane copy (a prefix cache reads 2)
+    hit, fetched = _down(oracle_mod, 64, [(0, 1, 3, 0), (0, 1, 5, 1)])
+    assert list(hit) == [0, 0] and fetched == 8
+    _, _, fetched_p = oracle_mod.cache_sim_prefix(1, 8, 64, [0, 0], [1, 1], [3, 5], [0, 1])
+    assert fetched_p == 5
+
+
+def test_downward_reuse_evicts_whole_lru_objects(oracle_mod):
+    # capacity 6: A(3) then B(2); C(3) needs room -> A (least recent) goes entirely
+    hit, fetched = _down(oracle_mod, 6, [(0, 0, 3, 0), (0, 1, 2, 1), (0, 2, 3, 2), (0, 0, 1, 3)])
+    assert list(hit) == [0, 0, 0, 0] and fetched == 3 + 2 + 3 + 1
+    # a promotion frees its own old copy first: A(2) -> A(5) fits in 5 planes
+    hit, fetched = _down(oracle_mod, 5, [(0, 0, 2, 0), (0, 0, 5, 1)])
+    assert list(hit) == [0, 0] and fetched == 7
+    # entries of the current batch are not evicted
+    with pytest.raises(ValueError):
+        _down(oracle_mod, 4, [(0, 0, 2, 0), (0, 1, 2, 0), (0, 2, 2, 0)])
+
+
+def test_downward_reuse_without_capacity_pressure_is_running_max(oracle_mod):
+    rng = np.random.default_rng(3)
+    L, E, n = 2, 16, 2000
+    lay = rng.integers(0, L, n)
+    exp_ = rng.integers(0, E, n)
+    dep = rng.integers(1, 9, n)
+    bat = np.arange(n)
+    hit, fetched = oracle_mod.cache_sim_independent_down(L, E, L * E * 8, lay, exp_, dep, bat)
+    best = {}
+    exp_hit, exp_fetched = [], 0
+    for l, e, b in zip(lay, exp_, dep):
+        r = best.get((l, e), 0)
+        exp_hit.append(1 if r >= b else 0)
+        if r < b:
+            exp_fetched += b
+            best[(l, e)] = b
+    assert list(hit) == exp_hit and fetched == exp_fetched
+    # exact-object hits are a subset of downward hits; a prefix cache fetches the least
+    hit_i, fetched_i = oracle_mod.cache_sim_independent(L, E, L * E * 8 * 8, lay, exp_, dep, bat)
+    assert np.all(hit >= hit_i)
+    _, _, fetched_p = oracle_mod.cache_sim_prefix(L, E, L * E * 8, lay, exp_, dep, bat)
+    assert fetched_p <= fetched <= fetched_i
