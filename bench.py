@@ -317,6 +317,7 @@ def cache_bench(args):
     stats = S.cache.stats().as_dict()
     lay, exp_, dep, bat = S.trace_arrays()
     hit_i, fetched_i = pm.cache_sim_independent(Lr, E, slots, lay, exp_, dep, bat)
+    hit_d, fetched_d = pm.cache_sim_independent_down(Lr, E, slots, lay, exp_, dep, bat)
     req_planes = int(dep.sum())
     t_half, st_half = marks[0]
     warm_tokens = T - (T // 2 + 1)           # tokens after the mid-run synchronisation
@@ -338,7 +339,10 @@ def cache_bench(args):
         "cache": {
             "requests": stats["requests"], "prefix_hit_rate": stats["hits"] / max(stats["requests"], 1),
             "independent_hit_rate": float(hit_i.mean()),
+            "downward_reuse_hit_rate": float(hit_d.mean()),
             "prefix_planes_fetched": stats["planes_fetched"], "independent_planes_fetched": fetched_i,
+            "downward_reuse_planes_fetched": fetched_d,
+            "downward_reuse_byte_hit_rate": 1.0 - fetched_d / max(req_planes, 1),
             "planes_requested": req_planes,
             "prefix_byte_hit_rate": 1.0 - stats["planes_fetched"] / max(req_planes, 1),
             "independent_byte_hit_rate": 1.0 - fetched_i / max(req_planes, 1),

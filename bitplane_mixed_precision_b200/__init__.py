@@ -73,6 +73,7 @@ _SIGS = {
     "pmoe_cache_eviction_log": ([P, P, i64, ctypes.POINTER(i64)], i32),
     "pmoe_cache_destroy": ([P], i32),
     "pmoe_cache_sim_independent": ([i32, i32, i64, i64, P, P, P, P, P, ctypes.POINTER(i64)], i32),
+    "pmoe_cache_sim_independent_down": ([i32, i32, i64, i64, P, P, P, P, P, ctypes.POINTER(i64)], i32),
     "pmoe_route_host": ([P, i32, i32, i32, P, P], i32),
     "pmoe_residual_norm": ([P, P, i32, i32, P, P], i32),
 }
@@ -308,6 +309,21 @@ def cache_sim_independent(layers, experts, cap_planes, layer, expert, need, batc
     hit = np.zeros(len(layer), dtype=np.uint8)
     fetched = i64(0)
     _check("pmoe_cache_sim_independent", _lib.pmoe_cache_sim_independent(
+        layers, experts, cap_planes, len(layer), _ptr(layer), _ptr(expert), _ptr(need), _ptr(batch),
+        _ptr(hit), ctypes.byref(fetched)))
+    return hit, fetched.value
+
+
+def cache_sim_independent_down(layers, experts, cap_planes, layer, expert, need, batch):
+    """Independent objects with downward reuse on a trace: (hit uint8 [n], planes_fetched)."""
+    import numpy as np
+    layer = np.ascontiguousarray(layer, dtype=np.int32)
+    expert = np.ascontiguousarray(expert, dtype=np.int32)
+    need = np.ascontiguousarray(need, dtype=np.uint8)
+    batch = np.ascontiguousarray(batch, dtype=np.int64)
+    hit = np.zeros(len(layer), dtype=np.uint8)
+    fetched = i64(0)
+    _check("pmoe_cache_sim_independent_down", _lib.pmoe_cache_sim_independent_down(
         layers, experts, cap_planes, len(layer), _ptr(layer), _ptr(expert), _ptr(need), _ptr(batch),
         _ptr(hit), ctypes.byref(fetched)))
     return hit, fetched.value

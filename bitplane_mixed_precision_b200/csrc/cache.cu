@@ -391,6 +391,62 @@ pmoe_status pmoe_cache_sim_independent(int layers, int experts, int64_t cap_plan
     return rc;
 }
 
+pmoe_status pmoe_cache_sim_independent_down(int layers, int experts, int64_t cap_planes, int64_t n,
+                                            const int32_t *layer, const int32_t *expert, const uint8_t *need,
+                                            const int64_t *batch, uint8_t *hit, int64_t *planes_fetched)
+{
+    if (layers <= 0 || experts <= 0 || cap_planes <= 0 || n < 0 || !planes_fetched ||
+        (n > 0 && (!layer || !expert || !need || !batch || !hit)))
+        return PMOE_ERR_INVALID_ARG;
+    for (int64_t a = 0; a < n; ++a)
+        if (layer[a] < 0 || layer[a] >= layers || expert[a] < 0 || expert[a] >= experts || need[a] < 1 ||
+            need[a] > 8)
+            return PMOE_ERR_INVALID_ARG;
+    // one copy per (layer, expert): its depth, last use and batch; LRU set of resident copies
+    const int64_t NE = (int64_t)layers * experts;
+    std::vector<uint8_t> depth(NE, 0);
+    std::vector<int64_t> last(NE, 0), obj_batch(NE, 0);
+    std::set<std::pair<int64_t, int64_t>> lru;
+    int64_t used = 0, fetched = 0;
+    pmoe_status rc = PMOE_OK;
+    for (int64_t a = 0; a < n && rc == PMOE_OK; ++a) {
+        const int b = need[a];
+        const int64_t x = (int64_t)layer[a] * experts + expert[a];
+        obj_batch[x] = batch[a];
+        if (depth[x] > 0)
+            lru.erase({last[x], x});
+        last[x] = a;
+        if (depth[x] >= b) {
+            hit[a] = 1;
+            lru.insert({a, x});
+            continue;
+        }
+        hit[a] = 0;
+        used -= depth[x]; // promotion replaces the old copy
+        depth[x] = 0;
+        while (used + b > cap_planes) {
+            auto it = lru.begin();
+            while (it != lru.end() && obj_batch[it->second] == batch[a])
+                ++it;
+            if (it == lru.end()) {
+                rc = PMOE_ERR_OUT_OF_SLOTS;
+                break;
+            }
+            used -= depth[it->second];
+            depth[it->second] = 0;
+            lru.erase(it);
+        }
+        if (rc != PMOE_OK)
+            break;
+        depth[x] = (uint8_t)b;
+        lru.insert({a, x});
+        used += b;
+        fetched += b;
+    }
+    *planes_fetched = fetched;
+    return rc;
+}
+
 pmoe_status pmoe_route_host(const float *logits, int T, int E, int k, int32_t *ids, float *w)
 {
     if (!logits || !ids || !w || T < 0 || k < 1 || k > 32 || E < k || E > 4096)

@@ -384,6 +384,20 @@ PMOE_API pmoe_status pmoe_cache_sim_independent(int layers, int experts, int64_t
                                                 int64_t *planes_fetched);
 
 /*
+ * pmoe_cache_sim_independent_down [T#51]: the independent design with
+ * downward reuse, host only: one copy per (layer, expert) at some depth r; an
+ * access at depth b hits when r >= b (the deeper copy serves it); otherwise a
+ * whole copy of b planes is loaded and replaces the old one (copies share no
+ * bits). Whole copies are evicted least-recently-used first (not those of the
+ * current batch) within cap_planes. Arguments and errors as
+ * pmoe_cache_sim_independent.
+ */
+PMOE_API pmoe_status pmoe_cache_sim_independent_down(int layers, int experts, int64_t cap_planes, int64_t n,
+                                                     const int32_t *layer, const int32_t *expert,
+                                                     const uint8_t *need, const int64_t *batch, uint8_t *hit,
+                                                     int64_t *planes_fetched);
+
+/*
  * pmoe_route_host: pmoe_route on host pointers (synchronous), for callers
  * that plan cache top-ups before launching the layer: ids (ties to the lower
  * id, larger logits first) and softmax weights in double rounded to float.

@@ -163,3 +163,27 @@ def test_route_host_matches_oracle(oracle_mod, synth_mod):
     w1 = np.zeros((1, 3), np.float32)
     pm.route_host(tied, 1, 8, 3, ids1, w1)
     assert list(ids1[0]) == [2, 5, 6]
+
+
+@pytest.mark.parametrize("seed,cap_frac", [(0, 0.3), (1, 0.12), (2, 0.5)])
+def test_downward_reuse_simulator_matches_oracle(oracle_mod, seed, cap_frac):
+    L, E = 3, 32
+    lay, exp_, dep, bat = _trace(seed + 20, L, E, 60, 6, zipf=True)
+    cap = max(int(cap_frac * L * E * 8), 8 * 6 * L)  # a token pins up to L layers x 6 experts x 8 planes
+    hit_o, fetched_o = oracle_mod.cache_sim_independent_down(L, E, cap, lay, exp_, dep, bat)
+    hit_p, fetched_p = pm.cache_sim_independent_down(L, E, cap, lay, exp_, dep, bat)
+    assert np.array_equal(hit_p, hit_o)
+    assert fetched_p == fetched_o
+
+
+def test_prefix_cache_bounds_downward_reuse(oracle_mod):
+    # with ample capacity: exact-object hits <= downward-reuse hits <= prefix hits, and the
+    # prefix cache fetches the fewest planes
+    L, E = 2, 16
+    lay, exp_, dep, bat = _trace(7, L, E, 80, 4, zipf=True)
+    cap = L * E * 8 * 8
+    _, _, st = _run_product(L, E, L * E * 8, lay, exp_, dep, bat, 4)
+    hit_d, fetched_d = pm.cache_sim_independent_down(L, E, cap, lay, exp_, dep, bat)
+    hit_i, fetched_i = pm.cache_sim_independent(L, E, cap, lay, exp_, dep, bat)
+    assert int(hit_i.sum()) <= int(hit_d.sum()) <= st.hits
+    assert st.planes_fetched <= fetched_d <= fetched_i
