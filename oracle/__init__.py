@@ -56,6 +56,7 @@ def _l():
             "or_cache_sim_prefix": ([i32, i32, i64, i64, P, P, P, P, P, P, i64, P, P], i32),
             "or_cache_sim_independent": ([i32, i32, i64, i64, P, P, P, P, P, P], i32),
             "or_cache_sim_independent_down": ([i32, i32, i64, i64, P, P, P, P, P, P], i32),
+            "or_select_cache_aware": ([P, P, P, P, i32, i32, i32, P], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -164,6 +165,21 @@ def select(w: np.ndarray, ids: np.ndarray, sens: np.ndarray, avg_bits: float) ->
     rc = _l().or_select(_p(w), _p(ids), _p(sens), T, k, avg_bits, _p(out))
     if rc:
         raise ValueError("or_select: bad arguments")
+    return out
+
+
+def select_cache_aware(w: np.ndarray, ids: np.ndarray, sens: np.ndarray, resident: np.ndarray,
+                       fetch: int) -> np.ndarray:
+    """Depths under a budget of fetched planes per token, resident planes free."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    sens = np.ascontiguousarray(sens, dtype=np.float32)
+    resident = np.ascontiguousarray(resident, dtype=np.uint8)
+    T, k = w.shape
+    out = np.empty((T, k), dtype=np.uint8)
+    rc = _l().or_select_cache_aware(_p(w), _p(ids), _p(sens), _p(resident), T, k, int(fetch), _p(out))
+    if rc:
+        raise ValueError("or_select_cache_aware: bad arguments")
     return out
 
 

@@ -659,3 +659,56 @@ int or_cache_sim_independent_down(int L, int E, int64_t cap_planes, int64_t n_ac
     free(last_batch);
     return rc;
 }
+
+/*
+ * Cache-aware prefix selection [T#61]: the cache-oblivious allocator budgets
+ * requested bits; this one budgets planes that must be fetched. Per token,
+ * with r_i the resident depth of slot i's expert (0..8):
+ *   b_i starts at max(1, r_i): resident planes cost no I/O, and every expert
+ *   needs at least its first plane (a fetch when r_i = 0);
+ *   then, while fewer than `fetch` planes have been fetched, the slot with the
+ *   largest w_i*s_e*2^-b_i among b_i < 8 (ties to the lower slot, exact
+ *   ldexpf) gets one more plane, each costing one fetch.
+ * This minimises sum w_i^2 s_e^2 4^-b_i under the fetch budget, because each
+ * further plane of a slot helps less than the one before.
+ */
+int or_select_cache_aware(const float *w, const int32_t *ids, const float *sens, const uint8_t *resident,
+                          int T, int k, int fetch, uint8_t *depth)
+{
+    if (T < 0 || k <= 0 || k > 64 || fetch < 0)
+        return 1;
+    float v[64];
+    int b[64];
+    for (int t = 0; t < T; ++t) {
+        int used = 0;
+        for (int i = 0; i < k; ++i) {
+            int r = resident[(size_t)t * k + i];
+            if (r > 8)
+                r = 8;
+            v[i] = w[(size_t)t * k + i] * sens[ids[(size_t)t * k + i]];
+            b[i] = r > 0 ? r : 1;
+            if (r == 0)
+                used += 1;
+        }
+        while (used < fetch) {
+            int best = -1;
+            float bestp = 0.0f;
+            for (int i = 0; i < k; ++i) {
+                if (b[i] >= 8)
+                    continue;
+                float pr = ldexpf(v[i], -b[i]);
+                if (best < 0 || pr > bestp) {
+                    best = i;
+                    bestp = pr;
+                }
+            }
+            if (best < 0)
+                break;
+            b[best] += 1;
+            used += 1;
+        }
+        for (int i = 0; i < k; ++i)
+            depth[(size_t)t * k + i] = (uint8_t)b[i];
+    }
+    return 0;
+}

@@ -168,3 +168,44 @@ def test_moe_layer_against_numpy(oracle_mod, synth_mod):
             h = g / (1 + np.exp(-g)) * u
             ref += float(w[t, i]) * (Wd @ h)
         np.testing.assert_allclose(y[t], ref, rtol=1e-10, atol=1e-13)
+
+
+@pytest.mark.parametrize("k", [1, 2, 3, 4])
+def test_cache_aware_select_is_brute_force_optimum(oracle_mod, k):
+    """Under a budget of fetched planes (resident planes free, every expert at least one plane),
+    the greedy reaches the exhaustive minimum of sum w^2 s^2 4^-b (transcript cue 61)."""
+    rng = np.random.default_rng(100 + k)
+    for trial in range(40):
+        w = rng.dirichlet(np.ones(k)).astype(np.float32)[None, :]
+        ids = np.arange(k, dtype=np.int32)[None, :]
+        sens = np.exp(0.5 * rng.standard_normal(k)).astype(np.float32)
+        res = rng.integers(0, 9, k).astype(np.uint8)
+        fetch = int(rng.integers(0, 3 * k + 1))
+        d = oracle_mod.select_cache_aware(w, ids, sens, res[None, :], fetch)[0]
+
+        def fetched(b):
+            return sum(max(0, int(bi) - int(ri)) for bi, ri in zip(b, res))
+        need = sum(1 for r in res if r == 0)
+        cap = max(fetch, need)
+        assert fetched(d) <= cap
+        assert all(int(bi) >= max(1, int(ri)) for bi, ri in zip(d, res))
+        best = math.inf
+        for cand in itertools.product(range(1, 9), repeat=k):
+            if fetched(cand) <= cap:
+                best = min(best, _objective(w[0], sens, cand))
+        assert _objective(w[0], sens, d) == pytest.approx(best, rel=1e-12)
+
+
+def test_cache_aware_select_special_cases(oracle_mod):
+    w = np.array([[0.5, 0.3, 0.2]], np.float32)
+    ids = np.array([[0, 1, 2]], np.int32)
+    sens = np.ones(3, np.float32)
+    # nothing resident: with a budget of k*B-style fetches it is the cache-oblivious greedy
+    d = oracle_mod.select_cache_aware(w, ids, sens, np.zeros((1, 3), np.uint8), 8)
+    assert np.array_equal(d, oracle_mod.select(w, ids, sens, 8 / 3))
+    # everything resident deeply, no fetch budget: all resident planes are used, nothing fetched
+    d = oracle_mod.select_cache_aware(w, ids, sens, np.array([[6, 3, 8]], np.uint8), 0)
+    assert list(d[0]) == [6, 3, 8]
+    # a zero budget still gives an absent expert its first plane
+    d = oracle_mod.select_cache_aware(w, ids, sens, np.array([[0, 2, 0]], np.uint8), 0)
+    assert list(d[0]) == [1, 2, 1]
