@@ -319,6 +319,25 @@ def cache_bench(args):
     hit_i, fetched_i = pm.cache_sim_independent(Lr, E, slots, lay, exp_, dep, bat)
     hit_d, fetched_d = pm.cache_sim_independent_down(Lr, E, slots, lay, exp_, dep, bat)
     req_planes = int(dep.sum())
+    # the same tokens again from a cold cache with cache-aware selection (resident planes free,
+    # the fetch budget of each token-layer = what the cache-oblivious depths fetch)
+    surrogate_oblivious = S.surrogate[1]
+    S.reset_cache()
+    S.cache_aware = True
+    torch.cuda.synchronize()
+    t_aw = time.perf_counter()
+    for t in range(T):
+        r.copy_(emb[t], non_blocking=True)
+        pm.residual_norm(r, None, 1, H, x, st)
+        S.decode_token(logits[t], r, x, y, t, stream=st)
+    torch.cuda.synchronize()
+    wall_aw = time.perf_counter() - t_aw
+    stats_aw = S.cache.stats().as_dict()
+    lay_aw, exp_aw, dep_aw, _ = S.trace_arrays()
+    aware = {"tokens_per_s": T / wall_aw, "prefix_hit_rate": stats_aw["hits"] / max(stats_aw["requests"], 1),
+             "planes_fetched": stats_aw["planes_fetched"], "planes_read": int(dep_aw.sum()),
+             "error_surrogate": S.surrogate[1], "error_surrogate_cache_oblivious": surrogate_oblivious,
+             "h2d_bytes_per_token": stats_aw["bytes_fetched"] / T}
     t_half, st_half = marks[0]
     warm_tokens = T - (T // 2 + 1)           # tokens after the mid-run synchronisation
     warm_s = wall - (t_half - t_start)
@@ -351,7 +370,9 @@ def cache_bench(args):
             "planes_evicted": stats["planes_evicted"],
             "second_half_prefix_hit_rate": (stats["hits"] - st_half["hits"]) /
                                            max(stats["requests"] - st_half["requests"], 1),
+            "planes_read": req_planes,
         },
+        "cache_aware": aware,
         "layer_error": list(err),
         "gpu_launches": T * (Lr * 3 + 1),  # per layer prep + expert kernel + residual; plus page-table updates
     }

@@ -55,6 +55,7 @@ _SIGS = {
     "pmoe_extract_prefix": ([P, i64, i32, i32, i32, P, P], i32),
     "pmoe_route": ([P, i32, i32, i32, P, P, P], i32),
     "pmoe_select_prefix": ([P, P, P, i32, i32, f32, P, i32, P], i32),
+    "pmoe_select_prefix_cache_aware": ([P, P, P, P, i32, i32, i32, P], i32),
     "pmoe_expert_gemv": ([ctypes.POINTER(Matrix), i32, P, i32, P, P], i32),
     "pmoe_layer_workspace_bytes": ([i32, i32, i32, i32, i32], sz),
     "pmoe_moe_layer_fwd": ([ctypes.POINTER(Layer), P, P, P, P, i32, i32, P, P, sz, P], i32),
@@ -153,6 +154,12 @@ def route(logits, T, E, k, ids, w, stream=None) -> None:
 def select_prefix(w, ids, sens, T, k, avg_bits, depth, on_device=True, stream=None) -> None:
     _check("pmoe_select_prefix", _lib.pmoe_select_prefix(_ptr(w), _ptr(ids), _ptr(sens), T, k, avg_bits,
                                                          _ptr(depth), int(on_device), _stream(stream)))
+
+
+def select_prefix_cache_aware(w, ids, sens, resident, T, k, fetch_budget, depth) -> None:
+    """Host arrays; depths under a budget of fetched planes per token (resident planes free)."""
+    _check("pmoe_select_prefix_cache_aware", _lib.pmoe_select_prefix_cache_aware(
+        _ptr(w), _ptr(ids), _ptr(sens), _ptr(resident), T, k, int(fetch_budget), _ptr(depth)))
 
 
 def make_matrix(planes, plane_stride_words, scales, codebook, N, K, G) -> Matrix:

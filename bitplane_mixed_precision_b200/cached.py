@@ -24,12 +24,12 @@ import numpy as np
 import torch
 
 from . import Cache, make_layer, moe_layer_fwd, layer_workspace_bytes, residual_norm, route_host, \
-    select_prefix, layer_error
+    select_prefix, select_prefix_cache_aware, layer_error
 
 
 class CachedStack:
     def __init__(self, L, E, H, I, G, k, avg_bits, slots, backing_layers, sens, device="cuda",
-                 keep_log=False):
+                 keep_log=False, cache_aware=False):
         """backing_layers: ResidentLayers (device) whose planes back the layers, as a list or as
         (count, make) with make(b) building backing b on demand: layer l uses backing
         l % count (host planes, scales, codebooks). Each backing's device pool is copied to
@@ -62,6 +62,11 @@ class CachedStack:
                                   self.page_table[l * E * 8:(l + 1) * E * 8], self.scales[l % nb],
                                   self.codebooks[l % nb]) for l in range(L)]
         self.sens = [np.ascontiguousarray(s, dtype=np.float32) for s in sens]
+        # cache-aware selection (transcript cue 61): per token-layer, the planes the cache-oblivious
+        # depths would fetch are the budget, and resident planes come free
+        self.cache_aware = cache_aware
+        self.keep_log = keep_log
+        self.surrogate = [0.0, 0.0]  # sum of w^2 s^2 4^-b: cache-oblivious depths, depths used
         self.side = torch.cuda.Stream(dev)
         self.done = [torch.cuda.Event() for _ in range(L)]
         for e in self.done:  # torch creates the CUDA event at its first record; the library records it
@@ -83,16 +88,26 @@ class CachedStack:
         # trace of accesses, for the independent-precision comparison
         self.trace = []
 
+    def _select(self, l, ids, w, dep):
+        """Depths of layer l's slots (host arrays of one token); cache-aware when enabled."""
+        sens = self.sens[l % len(self.sens)]
+        select_prefix(w, ids, sens, 1, self.k, self.avg_bits, dep, on_device=False)
+        v2 = (w.astype(np.float64) * sens[ids].astype(np.float64)) ** 2
+        self.surrogate[0] += float(np.sum(v2 * 4.0 ** (-dep.astype(np.float64))))
+        if self.cache_aware:
+            res = self.cache.resident_depth(l)[ids].astype(np.uint8)
+            fetch = int(np.maximum(dep.astype(np.int64) - res, 0).sum())
+            select_prefix_cache_aware(w, ids, sens, res, 1, self.k, fetch, dep)
+        self.surrogate[1] += float(np.sum(v2 * 4.0 ** (-dep.astype(np.float64))))
+
     def plan(self, logits, t):
-        """Host routing and selection for all layers of token t (logits: float32 [L, E])."""
+        """Host routing for all layers of token t (logits: float32 [L, E]); returns the set."""
         s = self.ntok % 2
         if self.set_used[s]:
             self.set_free[s].synchronize()  # that set's device copies of two tokens ago are done
-        ids, w, dep = self.ids_h[s].numpy(), self.w_h[s].numpy(), self.dep_h[s].numpy()
+        ids, w = self.ids_h[s].numpy(), self.w_h[s].numpy()
         for l in range(self.L):
             route_host(np.ascontiguousarray(logits[l], dtype=np.float32), 1, self.E, self.k, ids[l], w[l])
-            select_prefix(w[l], ids[l], self.sens[l % len(self.sens)], 1, self.k, self.avg_bits, dep[l],
-                          on_device=False)
         return s
 
     def decode_token(self, logits, r, x, y, t, stream=None, y_out=None):
@@ -101,9 +116,10 @@ class CachedStack:
         y_out: optional device float [L, H] receiving each layer's y."""
         st = stream if stream is not None else torch.cuda.current_stream(self.dev)
         s = self.plan(logits, t)
-        ids, dep = self.ids_h[s].numpy(), self.dep_h[s].numpy()
+        ids, w, dep = self.ids_h[s].numpy(), self.w_h[s].numpy(), self.dep_h[s].numpy()
         after = self.token_done if self.token_done_valid else None
         for l in range(self.L):
+            self._select(l, ids[l], w[l], dep[l])
             self.cache.extend(l, ids[l], dep[l], t, side=self.side, after=after, done=self.done[l])
             for e, b in zip(ids[l], dep[l]):
                 self.trace.append((l, int(e), int(b), t))
@@ -124,6 +140,18 @@ class CachedStack:
         self.token_done_valid = True
         self.ntok += 1
         return s
+
+    def reset_cache(self):
+        """A cold cache over the same pool and host planes (device work must be finished)."""
+        torch.cuda.synchronize(self.dev)
+        self.cache.close()
+        self.cache = Cache(self.L, self.E, self.slots, self.slot_words, self.pool, self.page_table,
+                           keep_log=self.keep_log)
+        nb = len(self.host)
+        self.cache.set_host_planes([self.host[l % nb] for l in range(self.L)])
+        self.trace = []
+        self.surrogate = [0.0, 0.0]
+        self.token_done_valid = False
 
     def routing(self, s):
         """Host copies (ids, w, depth) of the token planned into set s."""

@@ -100,6 +100,43 @@ pmoe_status pmoe_route(const float *logits, int T, int E, int k, int32_t *ids, f
     return launch_status();
 }
 
+pmoe_status pmoe_select_prefix_cache_aware(const float *w, const int32_t *ids, const float *sens,
+                                           const uint8_t *resident, int T, int k, int fetch_budget,
+                                           uint8_t *depth)
+{
+    if (!w || !ids || !sens || !resident || !depth || T < 0 || k < 1 || k > 32 || fetch_budget < 0)
+        return PMOE_ERR_INVALID_ARG;
+    for (int t = 0; t < T; ++t) {
+        float v[32];
+        int b[32], fetched = 0;
+        for (int i = 0; i < k; ++i) {
+            const int r = resident[t * k + i] < 8 ? resident[t * k + i] : 8;
+            v[i] = w[t * k + i] * sens[ids[t * k + i]];
+            b[i] = r > 0 ? r : 1; // resident planes are free; the first plane is always needed
+            fetched += (r == 0) ? 1 : 0;
+        }
+        for (; fetched < fetch_budget; ++fetched) {
+            int best = -1;
+            float bp = 0.0f;
+            for (int i = 0; i < k; ++i) {
+                if (b[i] >= 8)
+                    continue;
+                const float pr = ldexpf(v[i], -b[i]);
+                if (best < 0 || pr > bp) {
+                    best = i;
+                    bp = pr;
+                }
+            }
+            if (best < 0)
+                break;
+            b[best] += 1;
+        }
+        for (int i = 0; i < k; ++i)
+            depth[t * k + i] = (uint8_t)b[i];
+    }
+    return PMOE_OK;
+}
+
 pmoe_status pmoe_select_prefix(const float *w, const int32_t *ids, const float *sens, int T, int k,
                                float avg_bits, uint8_t *depth, int on_device, pmoe_stream stream)
 {

@@ -146,6 +146,20 @@ PMOE_API pmoe_status pmoe_route(const float *logits, int T, int E, int k, int32_
 PMOE_API pmoe_status pmoe_select_prefix(const float *w, const int32_t *ids, const float *sens, int T, int k,
                                float avg_bits, uint8_t *depth, int on_device, pmoe_stream stream);
 
+/*
+ * pmoe_select_prefix_cache_aware [T#61]: the allocator budgeted in planes to
+ * fetch instead of bits requested. Per token, with resident[t*k+i] the depth
+ * already cached for slot i's expert: each slot starts at max(1, resident)
+ * (cached planes cost nothing; a slot with nothing cached needs its first
+ * plane, one fetch), then while fewer than fetch_budget planes are fetched,
+ * the slot with the largest w*s_e*2^-b below 8 bits (ties to the lower slot)
+ * gets one more plane. Host pointers, synchronous: w float [T*k], ids int32
+ * [T*k], sens float [E], resident uint8 [T*k], depth uint8 [T*k] out.
+ */
+PMOE_API pmoe_status pmoe_select_prefix_cache_aware(const float *w, const int32_t *ids, const float *sens,
+                                                    const uint8_t *resident, int T, int k, int fetch_budget,
+                                                    uint8_t *depth);
+
 /* ------------------------------------------------------------------ */
 /* Execution                                                           */
 /* ------------------------------------------------------------------ */

@@ -88,3 +88,16 @@ def test_workspace_queries(pm):
     assert 0 < a < b
     m = pm.materialise_workspace_bytes(1, 10, 512, 4096, 1024)
     assert m >= 10 * 3 * 4096 * 1024 * 2  # bf16 copies of the ten selected experts
+
+
+def test_cache_aware_select_matches_oracle(pm, oracle_mod):
+    rng = np.random.default_rng(11)
+    T, k, E = 64, 10, 512
+    w = rng.dirichlet(np.ones(k), size=T).astype(np.float32)
+    ids = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+    sens = np.exp(0.5 * rng.standard_normal(E)).astype(np.float32)
+    res = rng.integers(0, 9, (T, k)).astype(np.uint8)
+    for fetch in (0, 3, 10, 25, 80):
+        got = np.zeros((T, k), np.uint8)
+        pm.select_prefix_cache_aware(w, ids, sens, res, T, k, fetch, got)
+        assert np.array_equal(got, oracle_mod.select_cache_aware(w, ids, sens, res, fetch))

@@ -35,11 +35,12 @@ def stack_setup(synth_mod):
     return dev, backs, sens
 
 
-def _run(stack_setup, synth_mod, slots, tokens, keep_log=True):
+def _run(stack_setup, synth_mod, slots, tokens, keep_log=True, cache_aware=False):
     import bitplane_mixed_precision_b200 as pm
     from bitplane_mixed_precision_b200.cached import CachedStack
     dev, backs, sens = stack_setup
-    S = CachedStack(L, E, H, I, G, K, AVG, slots, backs, sens, device=dev, keep_log=keep_log)
+    S = CachedStack(L, E, H, I, G, K, AVG, slots, backs, sens, device=dev, keep_log=keep_log,
+                    cache_aware=cache_aware)
     logits = np.stack([synth_mod.ar1_logits(SEED, l, tokens, E) for l in range(L)], axis=1)  # [t, l, E]
     emb = [synth_mod.activation_f32(SEED, t, 99, H) for t in range(tokens)]
     r = torch.empty(H, dtype=torch.float32, device=dev)
@@ -136,3 +137,19 @@ def test_residual_norm_matches_numpy(stack_setup):
     xf = (x.cpu().numpy().astype(np.int32) << 16).astype(np.uint32).view(np.float32)
     ref = r2 / np.sqrt((r2 ** 2).mean(axis=1, keepdims=True))
     assert np.max(np.abs(xf - ref)) <= 2 ** -7 * np.max(np.abs(ref))
+
+
+def test_cache_aware_selection_runs_bitwise_and_lowers_the_error_surrogate(stack_setup, synth_mod, oracle_mod):
+    # transcript cue 61: resident planes are free bits; the fetch budget is what the cache-oblivious
+    # depths would have fetched
+    S, outs, refs, routes, logits, _ = _run(stack_setup, synth_mod, slots=64, tokens=10, cache_aware=True)
+    for t, (a, b) in enumerate(zip(outs, refs)):
+        assert torch.equal(a, b), f"token {t}"
+    assert S.surrogate[1] <= S.surrogate[0]
+    assert S.surrogate[1] < S.surrogate[0]  # some resident planes were used
+    dev, backs, sens = stack_setup
+    for t in range(3):
+        ids, w, dep = routes[t]
+        for l in range(L):
+            assert all(int(b) >= 1 for b in dep[l])
+    S.close()
