@@ -57,6 +57,9 @@ def _l():
             "or_cache_sim_independent": ([i32, i32, i64, i64, P, P, P, P, P, P], i32),
             "or_cache_sim_independent_down": ([i32, i32, i64, i64, P, P, P, P, P, P], i32),
             "or_select_cache_aware": ([P, P, P, P, i32, i32, i32, P], i32),
+            "or_isotonic_nonincreasing": ([P, i32], None),
+            "or_profile_repair": ([P, i32, P], None),
+            "or_select_table": ([P, P, P, i32, i32, ctypes.c_float, P], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -181,6 +184,46 @@ def select_cache_aware(w: np.ndarray, ids: np.ndarray, sens: np.ndarray, residen
     if rc:
         raise ValueError("or_select_cache_aware: bad arguments")
     return out
+
+
+def isotonic_nonincreasing(g) -> np.ndarray:
+    g = np.array(g, dtype=np.float64)
+    _l().or_isotonic_nonincreasing(_p(g), len(g))
+    return g
+
+
+def profile_repair(raw) -> np.ndarray:
+    """raw: [n][8] errors at depths 1..8 -> repaired table [n][8]."""
+    raw = np.ascontiguousarray(raw, dtype=np.float64)
+    out = np.empty_like(raw)
+    _l().or_profile_repair(_p(raw), raw.shape[0], _p(out))
+    return out
+
+
+def select_table(w: np.ndarray, ids: np.ndarray, table: np.ndarray, avg_bits: float) -> np.ndarray:
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    table = np.ascontiguousarray(table, dtype=np.float32)
+    T, k = w.shape
+    out = np.empty((T, k), dtype=np.uint8)
+    rc = _l().or_select_table(_p(w), _p(ids), _p(table), T, k, avg_bits, _p(out))
+    if rc:
+        raise ValueError("or_select_table: bad arguments")
+    return out
+
+
+def expert_profile(expert: "Expert", E: int, H: int, I: int, G: int, xs: np.ndarray) -> np.ndarray:
+    """Relative output error of one expert at depths 1..8 against depth 8, averaged over the rows
+    of xs (double); the dequantise-then-matvec layer with this expert alone at weight 1."""
+    errs = np.zeros(8)
+    need = {0: expert}
+    ids = np.zeros((xs.shape[0], 1), np.int32)
+    w = np.ones((xs.shape[0], 1), np.float32)
+    ref = moe_layer(need, E, H, I, G, ids, w, np.full((xs.shape[0], 1), 8, np.uint8), xs)
+    for b in range(1, 9):
+        y = moe_layer(need, E, H, I, G, ids, w, np.full((xs.shape[0], 1), b, np.uint8), xs)
+        errs[b - 1] = float(np.mean(np.sum((y - ref) ** 2, axis=1) / np.sum(ref ** 2, axis=1)))
+    return errs
 
 
 class Expert:

@@ -712,3 +712,90 @@ int or_select_cache_aware(const float *w, const int32_t *ids, const float *sens,
     }
     return 0;
 }
+
+/*
+ * Error profiles [T#29, T#31]: E_e(b) for b = 1..8, the relative output error
+ * of an expert at depth b. Greedy allocation is valid when each further bit
+ * helps less than the one before; profiles that break this are repaired by
+ * isotonic regression. Reading: the gains g_b = E(b) - E(b+1), b = 1..7, are
+ * replaced by their least-squares non-increasing fit (pool adjacent
+ * violators, equal weights), clamped at 0, and E is rebuilt from E(8) upward
+ * (E(8) kept): E(b) = E(b+1) + g_b.
+ */
+void or_isotonic_nonincreasing(double *g, int n)
+{
+    double val[16];
+    int cnt[16];
+    int m = 0;
+    for (int i = 0; i < n; ++i) {
+        val[m] = g[i];
+        cnt[m] = 1;
+        ++m;
+        while (m > 1 && val[m - 2] < val[m - 1]) { /* violation of non-increasing order: pool */
+            double v = (val[m - 2] * cnt[m - 2] + val[m - 1] * cnt[m - 1]) / (cnt[m - 2] + cnt[m - 1]);
+            cnt[m - 2] += cnt[m - 1];
+            val[m - 2] = v;
+            --m;
+        }
+    }
+    int i = 0;
+    for (int j = 0; j < m; ++j)
+        for (int c = 0; c < cnt[j]; ++c)
+            g[i++] = val[j];
+}
+
+void or_profile_repair(const double *raw, int n, double *table)
+{
+    for (int e = 0; e < n; ++e) {
+        const double *E = raw + (size_t)e * 8;
+        double g[7];
+        for (int b = 0; b < 7; ++b)
+            g[b] = E[b] - E[b + 1];
+        or_isotonic_nonincreasing(g, 7);
+        double *out = table + (size_t)e * 8;
+        out[7] = E[7];
+        for (int b = 6; b >= 0; --b)
+            out[b] = out[b + 1] + (g[b] > 0.0 ? g[b] : 0.0);
+    }
+}
+
+/*
+ * Prefix selection from a profile table [T#29]: as or_select, with the gain of
+ * giving slot i its (b+1)-th bit = w_i^2 * (E_e(b) - E_e(b+1)) computed in
+ * float ((w*w) * (E[b-1] - E[b]), table of floats [E][8], entry b-1 = E(b)).
+ * Largest gain first, ties to the lower slot, 8-bit slots skipped.
+ */
+int or_select_table(const float *w, const int32_t *ids, const float *table, int T, int k, float avg_bits,
+                    uint8_t *depth)
+{
+    if (T < 0 || k <= 0 || k > 64)
+        return 1;
+    int B = or_budget(k, avg_bits);
+    int b[64];
+    for (int t = 0; t < T; ++t) {
+        for (int i = 0; i < k; ++i)
+            b[i] = 1;
+        for (int step = 0; step < B - k; ++step) {
+            int best = -1;
+            float bestp = 0.0f;
+            for (int i = 0; i < k; ++i) {
+                if (b[i] >= 8)
+                    continue;
+                float wi = w[(size_t)t * k + i];
+                const float *E = table + (size_t)ids[(size_t)t * k + i] * 8;
+                float gain = E[b[i] - 1] - E[b[i]];
+                float pr = (wi * wi) * gain;
+                if (best < 0 || pr > bestp) {
+                    best = i;
+                    bestp = pr;
+                }
+            }
+            if (best < 0)
+                break;
+            b[best] += 1;
+        }
+        for (int i = 0; i < k; ++i)
+            depth[(size_t)t * k + i] = (uint8_t)b[i];
+    }
+    return 0;
+}

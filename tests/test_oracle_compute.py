@@ -209,3 +209,73 @@ def test_cache_aware_select_special_cases(oracle_mod):
     # a zero budget still gives an absent expert its first plane
     d = oracle_mod.select_cache_aware(w, ids, sens, np.array([[0, 2, 0]], np.uint8), 0)
     assert list(d[0]) == [1, 2, 1]
+
+
+# Profile-driven allocation (transcript cues 29-31): isotonic repair of error profiles and
+# greedy selection from a per-expert table.
+
+def test_isotonic_matches_library_regression(oracle_mod):
+    from sklearn.isotonic import IsotonicRegression
+    rng = np.random.default_rng(4)
+    for trial in range(50):
+        g = rng.standard_normal(7) * rng.choice([0.1, 1.0, 10.0])
+        got = oracle_mod.isotonic_nonincreasing(g)
+        ref = IsotonicRegression(increasing=False).fit_transform(np.arange(7), g)
+        assert np.allclose(got, ref, rtol=0, atol=1e-12)
+    assert list(oracle_mod.isotonic_nonincreasing([3.0, 1.0, 2.0])) == [3.0, 1.5, 1.5]
+
+
+def test_profile_repair_keeps_valid_profiles_and_fixes_others(oracle_mod):
+    good = np.array([[0.7, 0.35, 0.15, 0.06, 0.024, 0.0096, 0.0028, 0.0]])
+    assert np.allclose(oracle_mod.profile_repair(good), good, rtol=0, atol=1e-15)
+    bad = np.array([[0.7, 0.6, 0.15, 0.14, 0.02, 0.0096, 0.0028, 0.0]])  # gains 0.1 < 0.45: not convex
+    rep = oracle_mod.profile_repair(bad)[0]
+    gains = rep[:-1] - rep[1:]
+    assert np.all(np.diff(gains) <= 1e-15) and np.all(gains >= 0)
+    assert rep[7] == bad[0, 7] and rep[0] == pytest.approx(bad[0, 0])  # total drop is preserved
+
+
+def test_select_table_reduces_to_closed_form_profiles(oracle_mod, synth_mod):
+    # E_e(b) = s_e^2 4^-b gives the same depths as the closed-form allocator
+    E, k, T = 64, 8, 200
+    sens = synth_mod.sensitivities(9, 0, E)
+    table = (sens.astype(np.float64)[:, None] ** 2 * 4.0 ** -np.arange(1, 9)[None, :]).astype(np.float32)
+    logits = np.stack([synth_mod.router_logits(9, t, 0, E) for t in range(T)])
+    ids, w = oracle_mod.route(logits, k)
+    assert np.array_equal(oracle_mod.select_table(w, ids, table, 2.5), oracle_mod.select(w, ids, sens, 2.5))
+
+
+@pytest.mark.parametrize("k", [2, 3, 4])
+def test_select_table_is_brute_force_optimum(oracle_mod, k):
+    rng = np.random.default_rng(200 + k)
+    for trial in range(30):
+        w = rng.dirichlet(np.ones(k)).astype(np.float32)[None, :]
+        ids = np.arange(k, dtype=np.int32)[None, :]
+        gains = np.sort(rng.random((k, 7)))[:, ::-1] * rng.random((k, 1))  # non-increasing gains
+        table = np.concatenate([np.cumsum(gains[:, ::-1], axis=1)[:, ::-1], np.zeros((k, 1))], axis=1)
+        table = table.astype(np.float32)
+        avg = float(rng.choice([1.5, 2.5, 4.0]))
+        B = oracle_mod.budget(k, avg)
+        d = oracle_mod.select_table(w, ids, table, avg)[0]
+        assert int(d.sum()) == B
+        obj = lambda b: sum(float(w[0, i]) ** 2 * float(table[i, b[i] - 1]) for i in range(k))
+        best = min(obj(c) for c in itertools.product(range(1, 9), repeat=k) if sum(c) == B)
+        assert obj(d) == pytest.approx(best, rel=1e-5, abs=1e-12)
+
+
+def test_expert_profile_shape(oracle_mod, synth_mod):
+    # the full expert's relative output error: zero at 8 bits, falling with depth, and a few times
+    # the squared relative weight error sqrt(D_b) of one matrix (three quantised matrices compound)
+    H, I, G, E = 1024, 256, 128, 4
+    cb = oracle_mod.tree_codebook_f32()
+    codes, scales = [], []
+    for m, (n, kk) in enumerate(((I, H), (I, H), (H, I))):
+        s, c = oracle_mod.quantize(synth_mod.expert_weights(5, 0, 1, m, n, kk), G)
+        codes.append(c)
+        scales.append(s)
+    ex = oracle_mod.Expert(codes, scales, [cb] * 3)
+    xs = np.random.default_rng(0).standard_normal((10, H))
+    prof = oracle_mod.expert_profile(ex, E, H, I, G, xs)
+    assert prof[7] == 0.0 and np.all(np.diff(prof) < 0)
+    D = np.array([0.603, 0.373, 0.234, 0.149, 0.096, 0.063, 0.041]) ** 2
+    assert np.all(prof[:7] / D > 1.0) and np.all(prof[:7] / D < 4.0)
