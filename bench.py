@@ -569,6 +569,34 @@ def main():
     t_mat = variant(lambda i, st: pm.materialise_layer_fwd(R.layer, x[i], ids[i], wts[i], dep[i], T, K_TOP,
                                                            y[i], mws, mws_bytes, st))
     del mws
+    # allocators compared on the true output error against 8 bits (64 tokens, 2.5 bits each):
+    # closed-form sensitivities s_e^2 4^-b vs error profiles measured on 10 Gaussian inputs
+    from bitplane_mixed_precision_b200.profile import expert_profiles
+    t_prof = time.perf_counter()
+    xprof = torch.from_numpy(np.stack([synth.activation_bf16(SEED, 10_000_000 + i, 0, H)
+                                       for i in range(10)]).view(np.int16)).to(dev)
+    _, table = expert_profiles(R, xprof)
+    prof_s = time.perf_counter() - t_prof
+    table_d = torch.from_numpy(table).to(dev)
+    na = 64
+    dep_t = torch.empty(na, K_TOP, dtype=torch.uint8, device=dev)
+    pm.select_prefix_table(wts[:na], ids[:na], table_d, na, K_TOP, AVG, dep_t)
+    y_ref = torch.empty(na, H, dtype=torch.float32, device=dev)
+    y_a = torch.empty(na, H, dtype=torch.float32, device=dev)
+    errs = torch.zeros(2, dtype=torch.float32, device=dev)
+    dep8 = torch.full((na, K_TOP), 8, dtype=torch.uint8, device=dev)
+    for i in range(na):
+        pm.moe_layer_fwd(R.layer, x[i], ids[i], wts[i], dep8[i], T, K_TOP, y_ref[i], ws, ws_bytes, stream)
+    for a_i, dd in enumerate((dep[:na], dep_t)):
+        for i in range(na):
+            pm.moe_layer_fwd(R.layer, x[i], ids[i], wts[i], dd[i], T, K_TOP, y_a[i], ws, ws_bytes, stream)
+        pm.relative_error(y_a, y_ref, na, H, errs[a_i:], stream)
+    torch.cuda.synchronize()
+    e_closed, e_prof = [float(v) for v in errs.cpu()]
+    allocators = {"tokens": na, "rel_sq_error_closed_form": e_closed, "rel_sq_error_profiles": e_prof,
+                  "profile_seconds": prof_s,
+                  "mean_bits_closed_form": float(dep[:na].float().mean()),
+                  "mean_bits_profiles": float(dep_t.float().mean())}
     sel_planes = float(dep_h[:nv].sum(axis=1).mean()) * 3 * PLANE_BYTES
     variants = {
         "tokens": nv,
@@ -578,6 +606,7 @@ def main():
                        "bitplane_gbs": K_TOP * 4 * 3 * PLANE_BYTES / t_u4 / 1e9},
         "materialise_bf16_ablation": {"tokens_per_s": 1.0 / t_mat, "us_per_token": t_mat * 1e6,
                                       "direct_speedup": t_mat / t_sel},
+        "allocators": allocators,
     }
 
     if rank == 0:

@@ -56,6 +56,9 @@ _SIGS = {
     "pmoe_route": ([P, i32, i32, i32, P, P, P], i32),
     "pmoe_select_prefix": ([P, P, P, i32, i32, f32, P, i32, P], i32),
     "pmoe_select_prefix_cache_aware": ([P, P, P, P, i32, i32, i32, P], i32),
+    "pmoe_relative_error": ([P, P, i32, i32, P, P], i32),
+    "pmoe_profile_repair": ([P, i32, P], i32),
+    "pmoe_select_prefix_table": ([P, P, P, i32, i32, f32, P, i32, P], i32),
     "pmoe_expert_gemv": ([ctypes.POINTER(Matrix), i32, P, i32, P, P], i32),
     "pmoe_layer_workspace_bytes": ([i32, i32, i32, i32, i32], sz),
     "pmoe_moe_layer_fwd": ([ctypes.POINTER(Layer), P, P, P, P, i32, i32, P, P, sz, P], i32),
@@ -160,6 +163,19 @@ def select_prefix_cache_aware(w, ids, sens, resident, T, k, fetch_budget, depth)
     """Host arrays; depths under a budget of fetched planes per token (resident planes free)."""
     _check("pmoe_select_prefix_cache_aware", _lib.pmoe_select_prefix_cache_aware(
         _ptr(w), _ptr(ids), _ptr(sens), _ptr(resident), T, k, int(fetch_budget), _ptr(depth)))
+
+
+def relative_error(y, ref, T, H, err, stream=None) -> None:
+    _check("pmoe_relative_error", _lib.pmoe_relative_error(_ptr(y), _ptr(ref), T, H, _ptr(err), _stream(stream)))
+
+
+def profile_repair(raw, n, table) -> None:
+    _check("pmoe_profile_repair", _lib.pmoe_profile_repair(_ptr(raw), n, _ptr(table)))
+
+
+def select_prefix_table(w, ids, table, T, k, avg_bits, depth, on_device=True, stream=None) -> None:
+    _check("pmoe_select_prefix_table", _lib.pmoe_select_prefix_table(
+        _ptr(w), _ptr(ids), _ptr(table), T, k, avg_bits, _ptr(depth), int(on_device), _stream(stream)))
 
 
 def make_matrix(planes, plane_stride_words, scales, codebook, N, K, G) -> Matrix:

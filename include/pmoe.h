@@ -160,6 +160,30 @@ PMOE_API pmoe_status pmoe_select_prefix_cache_aware(const float *w, const int32_
                                                     const uint8_t *resident, int T, int k, int fetch_budget,
                                                     uint8_t *depth);
 
+/*
+ * Profile-driven allocation [T#29, T#31]. An expert's error profile E_e(b),
+ * b = 1..8, is its relative output error at depth b, measured offline on
+ * random Gaussian inputs; the allocator then grants bits by the profile's
+ * gains instead of the closed form s_e^2 4^-b.
+ *
+ * pmoe_relative_error: err[0] = mean over the T rows of
+ *   ||y_t - ref_t||^2 / ||ref_t||^2 (double sums, fixed order). Device
+ *   pointers: y, ref float [T*H], err float [1]. Async on the stream.
+ * pmoe_profile_repair (host, synchronous): raw float [n][8] (entry b-1 =
+ *   E(b)) -> table float [n][8]: the gains E(b)-E(b+1) are replaced by their
+ *   least-squares non-increasing fit (pool adjacent violators), clamped at 0,
+ *   and the profile is rebuilt from E(8) upward, so that greedy allocation
+ *   grants bit b+1 of an expert only after bit b.
+ * pmoe_select_prefix_table: as pmoe_select_prefix, with the gain of giving a
+ *   slot its (b+1)-th bit = (w*w) * (E_e(b) - E_e(b+1)) in float (ties to the
+ *   lower slot). table float [E][8] (host or device with on_device).
+ */
+PMOE_API pmoe_status pmoe_relative_error(const float *y, const float *ref, int T, int H, float *err,
+                                         pmoe_stream stream);
+PMOE_API pmoe_status pmoe_profile_repair(const float *raw, int n, float *table);
+PMOE_API pmoe_status pmoe_select_prefix_table(const float *w, const int32_t *ids, const float *table, int T, int k,
+                                              float avg_bits, uint8_t *depth, int on_device, pmoe_stream stream);
+
 /* ------------------------------------------------------------------ */
 /* Execution                                                           */
 /* ------------------------------------------------------------------ */

@@ -101,3 +101,22 @@ def test_cache_aware_select_matches_oracle(pm, oracle_mod):
         got = np.zeros((T, k), np.uint8)
         pm.select_prefix_cache_aware(w, ids, sens, res, T, k, fetch, got)
         assert np.array_equal(got, oracle_mod.select_cache_aware(w, ids, sens, res, fetch))
+
+
+def test_profile_repair_and_table_select_match_oracle(pm, oracle_mod):
+    rng = np.random.default_rng(12)
+    n = 64
+    raw = np.sort(rng.random((n, 8)) * rng.random((n, 1)), axis=1)[:, ::-1].copy()
+    raw[:, 7] = 0.0
+    raw[::3, 2] = raw[::3, 1]  # some profiles with a flat step (not convex)
+    raw = raw.astype(np.float32)
+    table = np.zeros_like(raw)
+    pm.profile_repair(raw, n, table)
+    ref = oracle_mod.profile_repair(raw.astype(np.float64))
+    assert np.allclose(table, ref, rtol=1e-6, atol=1e-9)
+    T, k = 100, 10
+    w = rng.dirichlet(np.ones(k), size=T).astype(np.float32)
+    ids = np.stack([rng.choice(n, k, replace=False) for _ in range(T)]).astype(np.int32)
+    got = np.zeros((T, k), np.uint8)
+    pm.select_prefix_table(w, ids, table, T, k, 2.5, got, on_device=False)
+    assert np.array_equal(got, oracle_mod.select_table(w, ids, table, 2.5))

@@ -153,3 +153,34 @@ def test_cache_aware_selection_runs_bitwise_and_lowers_the_error_surrogate(stack
         for l in range(L):
             assert all(int(b) >= 1 for b in dep[l])
     S.close()
+
+
+def test_profile_driven_allocation(stack_setup, synth_mod, oracle_mod):
+    """Error profiles measured on the GPU equal the oracle's (dequantise-then-matvec in double) on
+    the same 10 Gaussian inputs; selection from the table is the same on device, host and oracle."""
+    import bitplane_mixed_precision_b200 as pm
+    from bitplane_mixed_precision_b200.profile import expert_profiles
+    from gpu_common import OracleExperts
+    import synth
+    dev, backs, sens = stack_setup
+    R = backs[1]
+    xb = np.stack([synth.activation_bf16(SEED, 5000 + i, 0, H) for i in range(10)])
+    raw, table = expert_profiles(R, torch.from_numpy(xb.view(np.int16)).to(dev))
+    assert np.all(raw[:, 7] == 0.0)
+    ox = OracleExperts(SEED, H, I, G, layer=1)
+    x64 = synth.bf16_to_f32(xb).astype(np.float64)
+    for e in (0, 5, 11):
+        ref = oracle_mod.expert_profile(ox.get(e), E, H, I, G, x64)
+        assert np.allclose(raw[e, :7], ref[:7], rtol=0.03), (e, raw[e], ref)
+    assert np.allclose(table, oracle_mod.profile_repair(raw.astype(np.float64)), rtol=1e-5, atol=1e-9)
+    T = 64
+    logits = np.stack([synth_mod.router_logits(SEED, t, 1, E) for t in range(T)])
+    ids, w = oracle_mod.route(logits, K)
+    host = np.zeros((T, K), np.uint8)
+    pm.select_prefix_table(w, ids, table, T, K, AVG, host, on_device=False)
+    devd = torch.empty(T, K, dtype=torch.uint8, device=dev)
+    pm.select_prefix_table(torch.from_numpy(w).to(dev), torch.from_numpy(ids).to(dev),
+                           torch.from_numpy(table).to(dev), T, K, AVG, devd)
+    torch.cuda.synchronize()
+    assert np.array_equal(devd.cpu().numpy(), host)
+    assert np.array_equal(host, oracle_mod.select_table(w, ids, table, AVG))
