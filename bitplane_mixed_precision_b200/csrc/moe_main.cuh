@@ -400,6 +400,127 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
     const int64_t mat_words = (int64_t)H * I / 32;
     const int64_t escale_len = 2 * (int64_t)I * (H / G) + (int64_t)H * (I / G);
     const bool stage_x = (T == 1 && H <= 4096);
+    // ---- producer state and item issue (warp NCW, lane 0 only)
+    int c = 0, pq = 0; // chunks and items the producer has issued
+    bool ok = true;
+    auto next_slot = [&](int &s) {
+        s = c % NSLOT;
+        if (c >= NSLOT && !pipe::mbar_wait(&S.empty[s], ((c / NSLOT) + 1) & 1, deadline)) {
+            set_error(W, kErrTimeout, 2);
+            ok = false;
+        }
+    };
+    auto make_desc = [&](int u) {
+        Desc d;
+        if (u >= total) {
+            d.kind = 2;
+            d.u = d.strip = 0;
+        } else if (u < totalA) {
+            d.kind = 0;
+            d.u = u / SA;
+            d.strip = u % SA;
+        } else {
+            d.kind = 1;
+            d.u = (u - totalA) / SB;
+            d.strip = (u - totalA) % SB;
+        }
+        d.c0 = c;
+        return d;
+    };
+    auto issue_item = [&](const UnitView &UV, const Desc &d) {
+        const int e = UV.expert(d.u), bmax = UV.bmax(d.u);
+        const int blk0 = UV.blk0(d.u), nblk = UV.nblk(d.u);
+        const float *esc = L.scales + (int64_t)e * escale_len;
+        // chunk order [planes | meta]: an item has at most 9 chunks, fewer than NSLOT, so none of
+        // its copies waits for a slot the item itself holds. A gate/up plane chunk holds the
+        // plane's 16 gate rows then its 16 up rows; a down plane chunk 128 rows of the down matrix.
+        auto issue_planes = [&]() {
+            for (int p = 0; p < bmax && ok; ++p) {
+                int s;
+                next_slot(s);
+                if (!ok)
+                    break;
+                const int slot = UV.slot(d.u, e, p);
+                const uint32_t bytes = d.kind == 0 ? (uint32_t)(2 * (H / 128) * 256) : (uint32_t)(8 * (I / 128) * 256);
+                if (slot >= 0) {
+                    const uint32_t *base = L.pool + (int64_t)slot * L.slot_words;
+                    pipe::mbar_arrive_expect_tx(&S.full[s], bytes);
+                    if (d.kind == 0) {
+                        const int64_t off = (int64_t)d.strip * (H / 128) * 64;
+                        pipe::bulk_g2s(S.ring[s], base + off, bytes / 2, &S.full[s]);
+                        pipe::bulk_g2s(S.ring[s] + bytes / 2, base + mat_words + off, bytes / 2, &S.full[s]);
+                    } else {
+                        pipe::bulk_g2s(S.ring[s], base + 2 * mat_words + (int64_t)d.strip * 8 * (I / 128) * 64,
+                                       bytes, &S.full[s]);
+                    }
+                } else {
+                    // a missing plane: report it and complete the slot without data
+                    set_error(W, kErrNoPlane, e * 8 + p);
+                    pipe::mbar_arrive(&S.full[s]);
+                }
+                ++c;
+            }
+        };
+        auto issue_meta = [&]() {
+            int s;
+            next_slot(s);
+            if (!ok)
+                return;
+            if (d.kind == 0) {
+                const uint32_t sb = 16 * (H / G) * 4;
+                pipe::mbar_arrive_expect_tx(&S.full[s], meta_bytes_gateup(H, G, nblk));
+                for (int m = 0; m < 2; ++m)
+                    pipe::bulk_g2s(S.ring[s] + m * sb,
+                                   esc + (int64_t)m * I * (H / G) + (int64_t)d.strip * 16 * (H / G), sb, &S.full[s]);
+                for (int bi = 0; bi < nblk; ++bi)
+                    for (int m = 0; m < 2; ++m)
+                        pipe::bulk_g2s(S.ring[s] + 2 * sb + (bi * 2 + m) * TAB_BYTES,
+                                       W.tabs + ((int64_t)(blk0 + bi) * 3 + m) * kTabWords, TAB_BYTES, &S.full[s]);
+            } else {
+                const uint32_t sb = 128 * (I / G) * 4;
+                int nmem = 0;
+                if (nblk == 1) {
+                    // the h fragments come along: wait (bounded) until the unit's h is converted
+                    nmem = UV.bnmem(blk0);
+                    while (pipe::ld_acquire(&W.readyB[d.u]) < I / 128) {
+                        if (pipe::globaltimer() > deadline) {
+                            set_error(W, kErrTimeout, 5);
+                            break;
+                        }
+                        __nanosleep(256);
+                    }
+                    pipe::fence_proxy_async();
+                }
+                pipe::mbar_arrive_expect_tx(&S.full[s], meta_bytes_down(I, G, nblk) + meta_bytes_down_frags(I, nmem));
+                pipe::bulk_g2s(S.ring[s], esc + 2 * (int64_t)I * (H / G) + (int64_t)d.strip * 128 * (I / G), sb,
+                               &S.full[s]);
+                for (int bi = 0; bi < nblk; ++bi)
+                    pipe::bulk_g2s(S.ring[s] + sb + bi * TAB_BYTES,
+                                   W.tabs + ((int64_t)(blk0 + bi) * 3 + 2) * kTabWords, TAB_BYTES, &S.full[s]);
+                unsigned char *fb = S.ring[s] + sb + nblk * TAB_BYTES;
+                for (int c2 = 0; c2 < nmem; ++c2) {
+                    const int pair = UV.bpair(blk0, c2);
+                    pipe::bulk_g2s(fb + c2 * 2 * I, W.hfrag + (int64_t)pair * (I / 32) * 16, 2 * I, &S.full[s]);
+                    pipe::bulk_g2s(fb + nmem * 2 * I + c2 * hexp_stride(I) * 4,
+                                   W.hexp + (int64_t)pair * hexp_stride(I), hexp_stride(I) * 4, &S.full[s]);
+                }
+            }
+            ++c;
+        };
+        issue_planes();
+        if (ok)
+            issue_meta();
+    };
+    // A gate/up first item is issued before the staging below, from the unit records in
+    // global memory, so that its copies are in flight while the CTA stages its tables.
+    if (warp == NCW && lane == 0 && (int)blockIdx.x < totalA) {
+        const UnitView VG{S, W, L.slot_of, false};
+        const Desc d = make_desc((int)blockIdx.x);
+        S.q[0] = d;
+        pipe::mbar_arrive(&S.qfull[0]);
+        pq = 1;
+        issue_item(VG, d);
+    }
     if (stage_x) {
         for (int i = tid; i < (H / 32) * 16; i += NTHREADS)
             S.xs[i] = W.xfrag[i];
@@ -426,125 +547,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
         // ------------------------------------------------------------ producer
         if (lane != 0)
             return;
-        int c = 0, qi = 0;
-        bool ok = true;
-        auto next_slot = [&](int &s) {
-            s = c % NSLOT;
-            if (c >= NSLOT && !pipe::mbar_wait(&S.empty[s], ((c / NSLOT) + 1) & 1, deadline)) {
-                set_error(W, kErrTimeout, 2);
-                ok = false;
-            }
-        };
         while (ok) {
             // claim only once the queue has room: an item is taken when this SM can start on it soon
-            const int qs = qi % QDEPTH;
-            if (qi >= QDEPTH && !pipe::mbar_wait(&S.qempty[qs], ((qi / QDEPTH) + 1) & 1, deadline)) {
+            const int qs = pq % QDEPTH;
+            if (pq >= QDEPTH && !pipe::mbar_wait(&S.qempty[qs], ((pq / QDEPTH) + 1) & 1, deadline)) {
                 set_error(W, kErrTimeout, 1);
                 break;
             }
-            Desc d;
             // the first item of each SM is its own index; the counter hands out the rest
-            const int u = (qi == 0) ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(&W.flags[kFlagSched], 1);
-            if (u >= total) {
-                d.kind = 2;
-                d.u = d.strip = 0;
-            } else if (u < totalA) {
-                d.kind = 0;
-                d.u = u / SA;
-                d.strip = u % SA;
-            } else {
-                d.kind = 1;
-                d.u = (u - totalA) / SB;
-                d.strip = (u - totalA) % SB;
-            }
-            d.c0 = c;
+            const int u = (pq == 0) ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(&W.flags[kFlagSched], 1);
+            const Desc d = make_desc(u);
             S.q[qs] = d;
             pipe::mbar_arrive(&S.qfull[qs]);
-            ++qi;
+            ++pq;
             if (d.kind == 2)
                 break;
-            const int e = V.expert(d.u), bmax = V.bmax(d.u);
-            const int blk0 = V.blk0(d.u), nblk = V.nblk(d.u);
-            const float *esc = L.scales + (int64_t)e * escale_len;
-            // chunk order [planes | meta]: an item has at most 9 chunks, fewer than NSLOT, so none of
-            // its copies waits for a slot the item itself holds. A gate/up plane chunk holds the
-            // plane's 16 gate rows then its 16 up rows; a down plane chunk 128 rows of the down matrix.
-            auto issue_planes = [&]() {
-                for (int p = 0; p < bmax && ok; ++p) {
-                    int s;
-                    next_slot(s);
-                    if (!ok)
-                        break;
-                    const int slot = V.slot(d.u, e, p);
-                    const uint32_t bytes = d.kind == 0 ? (uint32_t)(2 * (H / 128) * 256) : (uint32_t)(8 * (I / 128) * 256);
-                    if (slot >= 0) {
-                        const uint32_t *base = L.pool + (int64_t)slot * L.slot_words;
-                        pipe::mbar_arrive_expect_tx(&S.full[s], bytes);
-                        if (d.kind == 0) {
-                            const int64_t off = (int64_t)d.strip * (H / 128) * 64;
-                            pipe::bulk_g2s(S.ring[s], base + off, bytes / 2, &S.full[s]);
-                            pipe::bulk_g2s(S.ring[s] + bytes / 2, base + mat_words + off, bytes / 2, &S.full[s]);
-                        } else {
-                            pipe::bulk_g2s(S.ring[s], base + 2 * mat_words + (int64_t)d.strip * 8 * (I / 128) * 64,
-                                           bytes, &S.full[s]);
-                        }
-                    } else {
-                        // a missing plane: report it and complete the slot without data
-                        set_error(W, kErrNoPlane, e * 8 + p);
-                        pipe::mbar_arrive(&S.full[s]);
-                    }
-                    ++c;
-                }
-            };
-            auto issue_meta = [&]() {
-                int s;
-                next_slot(s);
-                if (!ok)
-                    return;
-                if (d.kind == 0) {
-                    const uint32_t sb = 16 * (H / G) * 4;
-                    pipe::mbar_arrive_expect_tx(&S.full[s], meta_bytes_gateup(H, G, nblk));
-                    for (int m = 0; m < 2; ++m)
-                        pipe::bulk_g2s(S.ring[s] + m * sb,
-                                       esc + (int64_t)m * I * (H / G) + (int64_t)d.strip * 16 * (H / G), sb, &S.full[s]);
-                    for (int bi = 0; bi < nblk; ++bi)
-                        for (int m = 0; m < 2; ++m)
-                            pipe::bulk_g2s(S.ring[s] + 2 * sb + (bi * 2 + m) * TAB_BYTES,
-                                           W.tabs + ((int64_t)(blk0 + bi) * 3 + m) * kTabWords, TAB_BYTES, &S.full[s]);
-                } else {
-                    const uint32_t sb = 128 * (I / G) * 4;
-                    int nmem = 0;
-                    if (nblk == 1) {
-                        // the h fragments come along: wait (bounded) until the unit's h is converted
-                        nmem = V.bnmem(blk0);
-                        while (pipe::ld_acquire(&W.readyB[d.u]) < I / 128) {
-                            if (pipe::globaltimer() > deadline) {
-                                set_error(W, kErrTimeout, 5);
-                                break;
-                            }
-                            __nanosleep(256);
-                        }
-                        pipe::fence_proxy_async();
-                    }
-                    pipe::mbar_arrive_expect_tx(&S.full[s], meta_bytes_down(I, G, nblk) + meta_bytes_down_frags(I, nmem));
-                    pipe::bulk_g2s(S.ring[s], esc + 2 * (int64_t)I * (H / G) + (int64_t)d.strip * 128 * (I / G), sb,
-                                   &S.full[s]);
-                    for (int bi = 0; bi < nblk; ++bi)
-                        pipe::bulk_g2s(S.ring[s] + sb + bi * TAB_BYTES,
-                                       W.tabs + ((int64_t)(blk0 + bi) * 3 + 2) * kTabWords, TAB_BYTES, &S.full[s]);
-                    unsigned char *fb = S.ring[s] + sb + nblk * TAB_BYTES;
-                    for (int c2 = 0; c2 < nmem; ++c2) {
-                        const int pair = V.bpair(blk0, c2);
-                        pipe::bulk_g2s(fb + c2 * 2 * I, W.hfrag + (int64_t)pair * (I / 32) * 16, 2 * I, &S.full[s]);
-                        pipe::bulk_g2s(fb + nmem * 2 * I + c2 * hexp_stride(I) * 4,
-                                       W.hexp + (int64_t)pair * hexp_stride(I), hexp_stride(I) * 4, &S.full[s]);
-                    }
-                }
-                ++c;
-            };
-            issue_planes();
-            if (ok)
-                issue_meta();
+            issue_item(V, d);
         }
         // no copy may still be landing in shared memory when the CTA exits
         for (int cc = (c > NSLOT ? c - NSLOT : 0); cc < c; ++cc)
