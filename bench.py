@@ -13,6 +13,10 @@ scaling); the path has no exchange step.
 
 --impl reference times the CPU oracle (the plain single-threaded C
 implementation) on a bounded sample of the same workload.
+
+Other workloads (their own JSON line): --workload batch (32-token batches with
+Zipf-biased routing, pairs grouped per expert) and --workload cache (16
+stacked layers decoding through the HBM prefix cache from pinned host planes).
 """
 from __future__ import annotations
 
