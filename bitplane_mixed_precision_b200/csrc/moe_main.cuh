@@ -11,7 +11,9 @@
 // rows of the item's matrices and the decode tables of its column blocks; for
 // down items of one column block also the members' h fragments). An item has
 // at most 9 chunks, fewer than the ring's slots, so no copy of an item ever
-// waits for a slot the same item still holds.
+// waits for a slot the same item still holds. An item's slots are free again
+// once the item is complete (its queue entry released), so consumers do not
+// release slots one by one.
 //
 // Consumers: every consumer warp takes every item and multiplies its share of
 // the item's tiles (gate/up: warps 0-7 the gate rows, 8-15 the up rows, each
@@ -60,7 +62,7 @@ struct Smem {
     uint32_t xs[XS_WORDS];
     uint32_t zeros[4];
     int xse[32];
-    uint64_t full[NSLOT], empty[NSLOT], qfull[QDEPTH], qempty[QDEPTH], epi[QDEPTH];
+    uint64_t full[NSLOT], qfull[QDEPTH], qempty[QDEPTH], epi[QDEPTH];
     Desc q[QDEPTH];
     int cnt[QDEPTH];
     UnitTab ut[UT_MAX];
@@ -378,7 +380,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
     if (tid == 0) {
         for (int s = 0; s < NSLOT; ++s) {
             pipe::mbar_init(&S.full[s], 1);
-            pipe::mbar_init(&S.empty[s], NCW);
         }
         for (int s = 0; s < QDEPTH; ++s) {
             pipe::mbar_init(&S.qfull[s], 1);
@@ -403,11 +404,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
     // ---- producer state and item issue (warp NCW, lane 0 only)
     int c = 0, pq = 0; // chunks and items the producer has issued
     bool ok = true;
+    // Ring slots are released per item, by the item's completion (its queue entry's qempty phase):
+    // a slot was last used by chunk c - NSLOT; every item before the previous one is complete once
+    // the current item has been claimed (the claim waits for the item QDEPTH back), so only a
+    // chunk of the previous item (first chunk prev_c0) has to wait, for that item to complete.
+    int prev_c0 = 0;
+    bool prev_done = true;
     auto next_slot = [&](int &s) {
         s = c % NSLOT;
-        if (c >= NSLOT && !pipe::mbar_wait(&S.empty[s], ((c / NSLOT) + 1) & 1, deadline)) {
-            set_error(W, kErrTimeout, 2);
-            ok = false;
+        if (c >= NSLOT && !prev_done && c - NSLOT >= prev_c0) {
+            const int n1 = pq - 2; // the previous item (pq already counts the current one)
+            if (!pipe::mbar_wait(&S.qempty[n1 % QDEPTH], (n1 / QDEPTH) & 1, deadline)) {
+                set_error(W, kErrTimeout, 2);
+                ok = false;
+            }
+            prev_done = true;
         }
     };
     auto make_desc = [&](int u) {
@@ -510,6 +521,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
         issue_planes();
         if (ok)
             issue_meta();
+        prev_c0 = d.c0;
+        prev_done = false;
     };
     // A gate/up first item is issued before the staging below, from the unit records in
     // global memory, so that its copies are in flight while the CTA stages its tables.
@@ -729,12 +742,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                 }
             }
             __syncwarp();
-            if (lane == 0)
-                for (int p = 0; p < bmax; ++p)
-                    pipe::mbar_arrive(&S.empty[(d.c0 + p) % NSLOT]);
-            __syncwarp();
-            if (lane == 0)
-                pipe::mbar_arrive(&S.empty[cm % NSLOT]);
             int last = 0;
             if (fast) {
                 // the epilogue warp reduces the partials; the last warp only hands the item over
@@ -836,11 +843,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                 }
             }
             __syncwarp();
-            if (lane == 0) {
-                for (int p = 0; p < bmax; ++p)
-                    pipe::mbar_arrive(&S.empty[(d.c0 + p) % NSLOT]);
-                pipe::mbar_arrive(&S.empty[cm % NSLOT]);
-            }
             int last = 0;
             if (fast) {
                 if (lane == 0) {
