@@ -17,15 +17,18 @@
 //
 // Consumers: every consumer warp takes every item and multiplies its share of
 // the item's tiles (gate/up: warps 0-7 the gate rows, 8-15 the up rows, each
-// an eighth of the columns). Partial sums go to a shared-memory slot of the item (one
-// slot per queue entry); the warp that finishes last (a shared-memory atomic)
-// reduces them in a fixed order, so results are deterministic, writes
-// h = silu(g) * u (gate/up) or the pair's output rows (down), and moves the
-// global counters: the last gate/up item of a 128-row tile of h converts it
-// to MMA fragments and bumps the unit's ready count; the last pair of a
-// token's 128 output rows sums the k pair outputs into y in slot order. Down
-// items wait (bounded) until their unit's h fragments are all ready. Items with
-// several column blocks (batched tokens) keep their partials in global memory.
+// an eighth of the columns). For items of one column block the partial sums go
+// to a shared-memory slot of the item (one per queue entry); the consumer warp
+// that finishes last (a shared-memory atomic) hands the item to the epilogue
+// warp, which reduces the partials in a fixed order, so results are
+// deterministic, releases the queue entry, then writes h = silu(g) * u
+// (gate/up) or the pair's output rows (down) and moves the global counters:
+// the last gate/up item of a 128-row tile of h converts it to MMA fragments and
+// bumps the unit's ready count; the last pair of a token's 128 output rows sums
+// the k pair outputs into y in slot order. Down items wait (bounded) until their
+// unit's h fragments are all ready. Items with several column blocks (batched
+// tokens) keep their partials in global memory, and the consumer warp that
+// finishes last (a global atomic) reduces them.
 namespace mk {
 
 constexpr int NCW = 16;                    // consumer warps
