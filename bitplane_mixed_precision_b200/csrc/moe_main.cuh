@@ -36,6 +36,9 @@ constexpr int NTHREADS = (NCW + 2) * 32; // + producer warp + epilogue warp
 constexpr int NSLOT = 12;                  // ring slots
 constexpr int CHUNK = 16384;               // bytes per ring slot
 constexpr int QDEPTH = 2;                  // item queue (= partial-sum slots): claim at most one item ahead
+// The producer's slot reuse waits only for the item before the current one: every older item is
+// complete once the current one is claimed, which holds for a two-entry queue.
+static_assert(QDEPTH == 2, "ring slot reuse assumes a two-entry item queue");
 constexpr int RED_WORDS = 16 * 4;          // per warp: [row][member]
 constexpr int XS_WORDS = (4096 / 32) * 16; // shared copy of the x fragments (T == 1, H <= 4096)
 constexpr int TAB_BYTES = 64;              // decode-table head copied per (block, matrix)
