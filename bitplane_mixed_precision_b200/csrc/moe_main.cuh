@@ -68,7 +68,7 @@ struct Smem {
     uint32_t xs[XS_WORDS];
     uint32_t zeros[4];
     int xse[32];
-    uint64_t full[NSLOT], qfull[QDEPTH], qempty[QDEPTH], epi[QDEPTH];
+    uint64_t ifull[QDEPTH], qfull[QDEPTH], qempty[QDEPTH], epi[QDEPTH]; // ifull: all of an item's bytes landed
     Desc q[QDEPTH];
     int cnt[QDEPTH];
     UnitTab ut[UT_MAX];
@@ -384,10 +384,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
     const uint64_t deadline = pipe::globaltimer() + kDeadlineNs;
 
     if (tid == 0) {
-        for (int s = 0; s < NSLOT; ++s) {
-            pipe::mbar_init(&S.full[s], 1);
-        }
         for (int s = 0; s < QDEPTH; ++s) {
+            pipe::mbar_init(&S.ifull[s], 1);
             pipe::mbar_init(&S.qfull[s], 1);
             pipe::mbar_init(&S.qempty[s], NCW + 1); // consumers + epilogue warp
             pipe::mbar_init(&S.epi[s], 1);
@@ -444,10 +442,25 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
         d.c0 = c;
         return d;
     };
-    auto issue_item = [&](const UnitView &UV, const Desc &d) {
+    int last_item = -1; // index of the last item whose copies were issued
+    auto issue_item = [&](const UnitView &UV, const Desc &d, int n) {
         const int e = UV.expert(d.u), bmax = UV.bmax(d.u);
         const int blk0 = UV.blk0(d.u), nblk = UV.nblk(d.u);
         const float *esc = L.scales + (int64_t)e * escale_len;
+        // all of the item's copies complete on its queue entry's barrier: one expect_tx with the
+        // item's bytes (planes present + meta), so that consumers wait once per item
+        uint64_t *bar = &S.ifull[n % QDEPTH];
+        {
+            const uint32_t pbytes = d.kind == 0 ? (uint32_t)(2 * (H / 128) * 256) : (uint32_t)(8 * (I / 128) * 256);
+            uint32_t total = d.kind == 0 ? (uint32_t)meta_bytes_gateup(H, G, nblk) : (uint32_t)meta_bytes_down(I, G, nblk);
+            if (d.kind == 1 && nblk == 1)
+                total += meta_bytes_down_frags(I, UV.bnmem(blk0));
+            for (int p = 0; p < bmax; ++p)
+                if (UV.slot(d.u, e, p) >= 0)
+                    total += pbytes;
+            pipe::mbar_arrive_expect_tx(bar, total);
+        }
+        last_item = n;
         // chunk order [planes | meta]: an item has at most 9 chunks, fewer than NSLOT, so none of
         // its copies waits for a slot the item itself holds. A gate/up plane chunk holds the
         // plane's 16 gate rows then its 16 up rows; a down plane chunk 128 rows of the down matrix.
@@ -461,19 +474,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                 const uint32_t bytes = d.kind == 0 ? (uint32_t)(2 * (H / 128) * 256) : (uint32_t)(8 * (I / 128) * 256);
                 if (slot >= 0) {
                     const uint32_t *base = L.pool + (int64_t)slot * L.slot_words;
-                    pipe::mbar_arrive_expect_tx(&S.full[s], bytes);
                     if (d.kind == 0) {
                         const int64_t off = (int64_t)d.strip * (H / 128) * 64;
-                        pipe::bulk_g2s(S.ring[s], base + off, bytes / 2, &S.full[s]);
-                        pipe::bulk_g2s(S.ring[s] + bytes / 2, base + mat_words + off, bytes / 2, &S.full[s]);
+                        pipe::bulk_g2s(S.ring[s], base + off, bytes / 2, bar);
+                        pipe::bulk_g2s(S.ring[s] + bytes / 2, base + mat_words + off, bytes / 2, bar);
                     } else {
                         pipe::bulk_g2s(S.ring[s], base + 2 * mat_words + (int64_t)d.strip * 8 * (I / 128) * 64,
-                                       bytes, &S.full[s]);
+                                       bytes, bar);
                     }
                 } else {
-                    // a missing plane: report it and complete the slot without data
+                    // a missing plane: report it (its bytes were not expected; the slot stays empty)
                     set_error(W, kErrNoPlane, e * 8 + p);
-                    pipe::mbar_arrive(&S.full[s]);
                 }
                 ++c;
             }
@@ -485,14 +496,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                 return;
             if (d.kind == 0) {
                 const uint32_t sb = 16 * (H / G) * 4;
-                pipe::mbar_arrive_expect_tx(&S.full[s], meta_bytes_gateup(H, G, nblk));
                 for (int m = 0; m < 2; ++m)
                     pipe::bulk_g2s(S.ring[s] + m * sb,
-                                   esc + (int64_t)m * I * (H / G) + (int64_t)d.strip * 16 * (H / G), sb, &S.full[s]);
+                                   esc + (int64_t)m * I * (H / G) + (int64_t)d.strip * 16 * (H / G), sb, bar);
                 for (int bi = 0; bi < nblk; ++bi)
                     for (int m = 0; m < 2; ++m)
                         pipe::bulk_g2s(S.ring[s] + 2 * sb + (bi * 2 + m) * TAB_BYTES,
-                                       W.tabs + ((int64_t)(blk0 + bi) * 3 + m) * kTabWords, TAB_BYTES, &S.full[s]);
+                                       W.tabs + ((int64_t)(blk0 + bi) * 3 + m) * kTabWords, TAB_BYTES, bar);
             } else {
                 const uint32_t sb = 128 * (I / G) * 4;
                 int nmem = 0;
@@ -508,18 +518,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                     }
                     pipe::fence_proxy_async();
                 }
-                pipe::mbar_arrive_expect_tx(&S.full[s], meta_bytes_down(I, G, nblk) + meta_bytes_down_frags(I, nmem));
                 pipe::bulk_g2s(S.ring[s], esc + 2 * (int64_t)I * (H / G) + (int64_t)d.strip * 128 * (I / G), sb,
-                               &S.full[s]);
+                               bar);
                 for (int bi = 0; bi < nblk; ++bi)
                     pipe::bulk_g2s(S.ring[s] + sb + bi * TAB_BYTES,
-                                   W.tabs + ((int64_t)(blk0 + bi) * 3 + 2) * kTabWords, TAB_BYTES, &S.full[s]);
+                                   W.tabs + ((int64_t)(blk0 + bi) * 3 + 2) * kTabWords, TAB_BYTES, bar);
                 unsigned char *fb = S.ring[s] + sb + nblk * TAB_BYTES;
                 for (int c2 = 0; c2 < nmem; ++c2) {
                     const int pair = UV.bpair(blk0, c2);
-                    pipe::bulk_g2s(fb + c2 * 2 * I, W.hfrag + (int64_t)pair * (I / 32) * 16, 2 * I, &S.full[s]);
+                    pipe::bulk_g2s(fb + c2 * 2 * I, W.hfrag + (int64_t)pair * (I / 32) * 16, 2 * I, bar);
                     pipe::bulk_g2s(fb + nmem * 2 * I + c2 * hexp_stride(I) * 4,
-                                   W.hexp + (int64_t)pair * hexp_stride(I), hexp_stride(I) * 4, &S.full[s]);
+                                   W.hexp + (int64_t)pair * hexp_stride(I), hexp_stride(I) * 4, bar);
                 }
             }
             ++c;
@@ -538,7 +547,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
         S.q[0] = d;
         pipe::mbar_arrive(&S.qfull[0]);
         pq = 1;
-        issue_item(VG, d);
+        issue_item(VG, d, 0);
     }
     if (stage_x) {
         for (int i = tid; i < (H / 32) * 16; i += NTHREADS)
@@ -581,11 +590,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
             ++pq;
             if (d.kind == 2)
                 break;
-            issue_item(V, d);
+            issue_item(V, d, pq - 1);
         }
-        // no copy may still be landing in shared memory when the CTA exits
-        for (int cc = (c > NSLOT ? c - NSLOT : 0); cc < c; ++cc)
-            pipe::mbar_wait(&S.full[cc % NSLOT], (cc / NSLOT) & 1, deadline + kDeadlineNs);
+        // no copy may still be landing in shared memory when the CTA exits: items before the last
+        // two are complete (their consumers finished), so wait for those two
+        for (int n = (last_item > 0 ? last_item - 1 : 0); n <= last_item; ++n)
+            pipe::mbar_wait(&S.ifull[n % QDEPTH], (n / QDEPTH) & 1, deadline + kDeadlineNs);
         return;
     }
 
@@ -689,7 +699,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
         bool fine = true;
         const int cm = d.c0 + bmax; // meta chunk (after the item's planes)
         const unsigned char *meta = S.ring[cm % NSLOT];
-        if (!pipe::mbar_wait(&S.full[cm % NSLOT], (cm / NSLOT) & 1, deadline))
+        if (!pipe::mbar_wait(&S.ifull[qs], (qi / QDEPTH) & 1, deadline)) // the item's bytes
             fine = false;
 
         if (d.kind == 0) {
@@ -703,8 +713,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
             for (int p = 0; p < 8; ++p) {
                 const int cc = d.c0 + p;
                 pp[p] = S.ring[cc % NSLOT] + tix0 * 256 + lane * 8;
-                if (p < bmax && !pipe::mbar_wait(&S.full[cc % NSLOT], (cc / NSLOT) & 1, deadline))
-                    fine = false;
             }
             {
                 const float *sc0 = reinterpret_cast<const float *>(meta) + (m * 16 + g) * ngr + Q0 * (128 / G);
@@ -804,8 +812,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
             for (int p = 0; p < 8; ++p) {
                 const int cc = d.c0 + p;
                 pp[p] = S.ring[cc % NSLOT] + tix0 * 256 + lane * 8;
-                if (p < bmax && !pipe::mbar_wait(&S.full[cc % NSLOT], (cc / NSLOT) & 1, deadline))
-                    fine = false;
             }
             const float *sc0 = reinterpret_cast<const float *>(meta) + (16 * sb + g) * ngr + Q0 * (128 / G);
             const float *sc1 = sc0 + 8 * ngr;
