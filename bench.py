@@ -85,6 +85,26 @@ def traffic_from_profiles():
     return None
 
 
+def max_over_ranks(t, world, device):
+    """The largest of the ranks' values of t, on every rank (t itself when world == 1). The ranks'
+    process group must be up; device is where the reduction runs (cuda for nccl, cpu for gloo)."""
+    if world == 1:
+        return t
+    import torch
+    import torch.distributed as dist
+    tt = torch.tensor([t], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def gpu_bus_id(dev):
+    """PCI bus id of a torch CUDA device, as nvidia-smi --id accepts it (its indices ignore
+    CUDA_VISIBLE_DEVICES)."""
+    import torch
+    pr = torch.cuda.get_device_properties(dev)
+    return f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+
+
 class ClockSampler:
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -476,7 +496,7 @@ def batch_bench(args):
     for g, _ in graphs[:1]:
         g.replay()
     torch.cuda.synchronize()
-    clk = ClockSampler(0)
+    clk = ClockSampler(gpu_bus_id(dev))
     clk.start()
     a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
@@ -616,8 +636,7 @@ def main():
         g.replay()
     torch.cuda.synchronize()
 
-    pr = torch.cuda.get_device_properties(dev)
-    clocks = ClockSampler(f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0")
+    clocks = ClockSampler(gpu_bus_id(dev))
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -633,11 +652,8 @@ def main():
     t_stop.record()
     torch.cuda.synchronize()
     clk = clocks.stop()
-    elapsed = t_start.elapsed_time(t_stop) * 1e-3
+    elapsed = max_over_ranks(t_start.elapsed_time(t_stop) * 1e-3, world, dev)
     if world > 1:
-        tt = torch.tensor([elapsed], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed = float(tt.item())
         dist.barrier()
     value = args.steps * world / elapsed
 
@@ -661,11 +677,7 @@ def main():
         y_pin[i].copy_(y_d, non_blocking=True)
     e1.record()
     torch.cuda.synchronize()
-    e2e_t = e0.elapsed_time(e1) * 1e-3
-    if world > 1:
-        tt = torch.tensor([e2e_t], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_t = float(tt.item())
+    e2e_t = max_over_ranks(e0.elapsed_time(e1) * 1e-3, world, dev)
     e2e = {"value": ne * world / e2e_t, "unit": "tokens/s", "h2d_bytes_per_step": E * 4 + H * 2,
            "d2h_bytes_per_step": H * 4}
 
