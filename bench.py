@@ -64,6 +64,15 @@ def workload(e):
     return f"moe_layer_e{e}_top10_h4096_i1024_g128_avg2.5_batch1"
 
 
+def layer_config(world):
+    """The config of the batch-1 layer workload (both arms report the same one)."""
+    return {"workload": workload(E), "experts": E, "top_k": K_TOP, "hidden": H, "inter": I,
+            "group": G, "avg_bits": AVG, "batch": 1, "tokens_distinct": N_TOKENS,
+            "parallelism": f"replicas x{world}",
+            "l2": f"inputs larger than L2 ({E * 3 * 8 * PLANE_BYTES / 1e9:.1f} GB of resident planes), "
+                  "fresh token per step; kernel timing with L2 flushed before each token"}
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -251,7 +260,7 @@ def reference_arm(args):
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / max(args.steps, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": workload(E)},
+            "data": "synthetic", "config": layer_config(1),
             "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                              "sample": f"per step: {rows} rows of one selected expert matrix at its "
                                        f"selected depth (dequantise-then-matvec in double); tokens "
@@ -769,11 +778,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": elapsed * 1e3 / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "s8 mma / s32 acc / f32",
             "data": "synthetic",
-            "config": {"workload": workload(E), "experts": E, "top_k": K_TOP, "hidden": H, "inter": I,
-                       "group": G, "avg_bits": AVG, "batch": 1, "tokens_distinct": N_TOKENS,
-                       "parallelism": f"replicas x{world}",
-                       "l2": f"inputs larger than L2 ({E * 3 * 8 * PLANE_BYTES / 1e9:.1f} GB of resident planes), fresh token per step; "
-                             "kernel timing with L2 flushed before each token"},
+            "config": layer_config(world),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "kernel": "moe_main_kernel (gate/up+SwiGLU, down, combine)",
