@@ -3,20 +3,23 @@
 // (token, expert) pairs by expert, gate/up prefix GEMV + SwiGLU, down prefix
 // GEMV and the routing-weighted combine.
 //
-// Two launches per call:
+// Launches per call:
+//  * xfrag_kernel, only when the batch is too large for the prep kernel to do
+//    it: the activations' MMA fragments.
 //  * layer_prep_kernel (one CTA): routing and selection (decode step), pairs
 //    grouped by expert into column blocks (<= 4 pairs of one depth) and units
-//    (<= 4 blocks of one expert, deepest units first), decode tables,
-//    activation fragments, and zeroed counters.
+//    (<= 4 blocks of one expert, deepest units first), one record per unit,
+//    decode tables, activation fragments (small batches) and zeroed counters.
 //  * moe_main_kernel (persistent, one CTA per SM, launched as a programmatic
-//    dependent of the prep kernel): one producer warp grabs work items from a
+//    dependent of the prep kernel): a producer warp claims work items from a
 //    global counter and streams their plane chunks into a shared-memory ring
-//    with 1-D bulk copies; 16 consumer warps decode and multiply. Gate/up
-//    items (unit, 32 rows of I) come first; each writes h = silu(g) * u, and
-//    the last one of a unit turns h into MMA fragments and sets the unit's
-//    ready flag. Down items (unit, 128 rows of H) wait for that flag, write
-//    each pair's output rows, and the last pair of a token row strip sums the
-//    k contributions in slot order into y.
+//    with 1-D bulk copies; 16 consumer warps decode and multiply; an epilogue
+//    warp finishes items of one column block. Gate/up items (unit, 16 rows of
+//    I) come first; each writes its rows of h = silu(g) * u, and the last one
+//    of a 128-row tile of h turns the tile into MMA fragments and counts it
+//    toward the unit's ready count. Down items (unit, 128 rows of H) wait for
+//    that count, write each pair's output rows, and the last pair of a token
+//    row strip sums the k contributions in slot order into y.
 // A plane chunk is read once per unit and decoded for every column block at
 // the block's own depth, so tokens at different depths of one expert share
 // the planes they have in common (transcript cues 13, 35).
