@@ -5,8 +5,9 @@
 // Producer: takes work items from a global counter (gate/up items first, then
 // down items; units deepest first), one at a time once the two-entry item
 // queue has room, publishes each item in that queue and streams the item's
-// bytes into a ring of 16 KB shared-memory slots with 1-D bulk copies
-// completing on mbarriers: one chunk per plane ([16 gate rows | 16 up rows] of
+// bytes into a ring of 16 KB shared-memory slots with 1-D bulk copies that
+// all complete on the item's mbarrier (one per queue entry, armed once with
+// the item's bytes): one chunk per plane ([16 gate rows | 16 up rows] of
 // a gate/up item, 128 rows of a down item) and then a "meta" chunk (the scale
 // rows of the item's matrices and the decode tables of its column blocks; for
 // down items of one column block also the members' h fragments). An item has
