@@ -1,6 +1,7 @@
 // Persistent expert kernel of the MoE layer (included by layer.cu).
 //
-// One CTA per SM: warp NCW is the producer, warps 0..NCW-1 consume.
+// One CTA per SM: warp NCW is the producer, warps 0..NCW-1 consume, warp NCW+1
+// is the epilogue warp.
 //
 // Producer: takes work items from a global counter (gate/up items first, then
 // down items; units deepest first), one at a time once the two-entry item
