@@ -35,11 +35,12 @@ namespace {
 constexpr int kStageBufs = 8;         // page-table update buffers in flight
 constexpr int kStageEntries = 16384;  // updates per buffer
 
-// Order of routing keys: larger float first, -0 below +0 (as the device routing's keys).
+// Order of routing keys: larger float first, -0 equal to +0 (as the device routing's keys).
 inline uint32_t ord_key_host(float f)
 {
     uint32_t u;
     std::memcpy(&u, &f, 4);
+    u = (u == 0x80000000u) ? 0u : u;
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 

@@ -8,10 +8,12 @@
 namespace pmoe {
 namespace dev {
 
-// Order-preserving map of float to uint32 (larger float -> larger key, > 0).
+// Order-preserving map of float to uint32 (larger float -> larger key, > 0);
+// -0 and +0 are equal logits and get the same key (a tie, to the lower id).
 __device__ __forceinline__ uint32_t ord_key(float f)
 {
-    const uint32_t u = __float_as_uint(f);
+    uint32_t u = __float_as_uint(f);
+    u = (u == 0x80000000u) ? 0u : u;
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
