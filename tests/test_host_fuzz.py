@@ -150,3 +150,17 @@ def test_cache_manager_matches_oracle_simulator(oracle_mod, trace, per_call):
     hit_od, fetched_d_o = oracle_mod.cache_sim_independent_down(L, E, cap, lay, exp_, dep, bat)
     hit_pd, fetched_d_p = pm.cache_sim_independent_down(L, E, cap, lay, exp_, dep, bat)
     assert np.array_equal(hit_pd, hit_od) and fetched_d_p == fetched_d_o
+
+
+@FUZZ
+@given(st.integers(1, 8), st.integers(1, 8), st.integers(1, 8), st.integers(0, 2**32 - 1))
+def test_host_pack_matches_oracle(oracle_mod, n16, k128, depth, seed):
+    N, K = 16 * n16, 128 * k128
+    rng = np.random.default_rng(seed)
+    codes = rng.integers(0, 256, size=(N, K), dtype=np.uint8)
+    stride = N * K // 32
+    out = np.zeros(stride * depth, dtype=np.uint32)
+    pm.pack_bitplanes(codes, N, K, depth, out, stride, on_device=False)
+    ref = oracle_mod.pack(codes, depth)
+    for p in range(depth):
+        assert np.array_equal(out[p * stride:(p + 1) * stride], ref[p])
