@@ -18,6 +18,8 @@ def _weights(rng, T, k, ties):
     w = rng.dirichlet(np.ones(k), size=T).astype(np.float32)
     if ties:
         w[:] = np.float32(1.0 / k)  # every slot equal: ties decide every step
+    elif k > 1 and rng.random() < 0.3:
+        w[:, rng.integers(0, k)] = 0.0  # a routing weight that underflowed to zero
     return w
 
 
