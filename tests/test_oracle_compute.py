@@ -279,3 +279,105 @@ def test_expert_profile_shape(oracle_mod, synth_mod):
     assert prof[7] == 0.0 and np.all(np.diff(prof) < 0)
     D = np.array([0.603, 0.373, 0.234, 0.149, 0.096, 0.063, 0.041]) ** 2
     assert np.all(prof[:7] / D > 1.0) and np.all(prof[:7] / D < 4.0)
+
+
+# The layer's composition (gate/up -> SwiGLU -> down -> weighted combine), pinned by cases whose
+# result follows from the definition by hand, not by re-running its formula: PagedMoE transcript
+# cue 4 (top-k experts combined with routing weights that sum to one) and the SwiGLU expert FFN.
+
+def _const_expert(oracle_mod, H, I, G, cb, codes_gud, scales_gud):
+    """An expert whose three matrices have one code and one scale each (all weights equal)."""
+    codes = [np.full(shape, c, np.uint8) for shape, c in zip(((I, H), (I, H), (H, I)), codes_gud)]
+    scales = [np.full((n, kk // G), s, np.float32)
+              for (n, kk), s in zip(((I, H), (I, H), (H, I)), scales_gud)]
+    return oracle_mod.Expert(codes, scales, [cb] * 3)
+
+
+def _ident_codebook():
+    """A 510-entry table whose every depth maps index 0 to 0.0 and the all-ones index to 1.0
+    (any other entry 0.5): code 0 reads as 0 and code 255 as 1 at every depth."""
+    cb = np.full(510, 0.5, np.float32)
+    for d in range(1, 9):
+        cb[(1 << d) - 2] = 0.0
+        cb[(1 << d) - 2 + (1 << d) - 1] = 1.0
+    return cb
+
+
+@pytest.mark.parametrize("b", [1, 3, 8])
+def test_layer_negative_gate_silences_the_expert(oracle_mod, b):
+    """Gate weights all at the most negative tree node, up weights all at the most positive one,
+    x > 0: g is a large negative number, silu(g) ~ 0, so the expert adds (almost) nothing.
+    With gate and up swapped (silu(u) * g) the output would be of order -u*g*H instead."""
+    H, I, G = 128, 128, 64
+    cb = oracle_mod.tree_codebook_f32()
+    ex = _const_expert(oracle_mod, H, I, G, cb, (0, 255, 255), (1.0, 1.0, 1.0))
+    x = np.full((1, H), 0.5)
+    y = oracle_mod.moe_layer({0: ex}, 1, H, I, G, np.zeros((1, 1), np.int32), np.ones((1, 1), np.float32),
+                             np.full((1, 1), b, np.uint8), x)
+    c_lo, c_hi = float(oracle_mod.level(cb, b)[0]), float(oracle_mod.level(cb, b)[-1])
+    g, u = c_lo * 0.5 * H, c_hi * 0.5 * H   # every row of Wg x and Wu x
+    assert g < -40 and u > 40
+    bound = abs(g) * math.exp(g) * u * c_hi * I * 1.01  # |silu(g)| <= |g| e^g for g < 0
+    assert np.all(np.abs(y) <= bound)
+    assert bound < 1e-10
+    swapped = (u / (1 + math.exp(-u))) * g * c_hi * I
+    assert abs(swapped) > 1e3
+
+
+def test_layer_identity_down_returns_swiglu(oracle_mod):
+    """Wg = a*I, Wu = c*I, Wd = I (codes 255 on the diagonal, 0 elsewhere, a table with 0 and 1
+    at its ends): y = w * silu(a x) * (c x) element by element, with a != c so that a swapped
+    gate/up gives another value. silu(z) = z * sigmoid(z) is checked at points with known values."""
+    H = I = 128
+    G = 64
+    cb = _ident_codebook()
+    a, c, wt = 1.5, -0.75, 0.625
+    eye = np.where(np.eye(H, dtype=bool), 255, 0).astype(np.uint8)
+    codes = [eye, eye, eye]
+    scales = [np.full((I, H // G), a, np.float32), np.full((I, H // G), c, np.float32),
+              np.full((H, I // G), 1.0, np.float32)]
+    ex = oracle_mod.Expert(codes, scales, [cb] * 3)
+    x = np.linspace(-3.0, 3.0, H)[None, :]
+    for b in (1, 2, 5, 8):
+        y = oracle_mod.moe_layer({0: ex}, 1, H, I, G, np.zeros((1, 1), np.int32),
+                                 np.full((1, 1), wt, np.float32), np.full((1, 1), b, np.uint8), x)[0]
+        g, u = a * x[0], c * x[0]
+        # sigmoid from tanh: sigma(z) = (1 + tanh(z/2)) / 2, another route to the same function
+        want = wt * g * (0.5 * (1.0 + np.tanh(0.5 * g))) * u
+        np.testing.assert_allclose(y, want, rtol=1e-12, atol=1e-15)
+        swapped = wt * u * (0.5 * (1.0 + np.tanh(0.5 * u))) * g
+        assert np.max(np.abs(swapped - want)) > 0.1
+    # silu at points with closed-form values: silu(0) = 0 and silu(2 ln 3) = ln 3 * 3/2 ... via x
+    x0 = np.zeros((1, H))
+    y0 = oracle_mod.moe_layer({0: ex}, 1, H, I, G, np.zeros((1, 1), np.int32), np.ones((1, 1), np.float32),
+                              np.full((1, 1), 8, np.uint8), x0)
+    assert np.all(y0 == 0.0)
+
+
+def test_layer_is_linear_in_routing_weights(oracle_mod, synth_mod):
+    """y = sum_i w_i * expert_i(x): splitting the weights into one-hot vectors and summing the
+    results reproduces the output (a weight applied before gate/up, where silu is not linear,
+    would break this)."""
+    E, k, H, I, G = 6, 3, 256, 128, 64
+    cb = oracle_mod.tree_codebook_f32()
+    experts = {}
+    for e in range(E):
+        codes, scales = [], []
+        for m, (n, kk) in enumerate(((I, H), (I, H), (H, I))):
+            s, cc = oracle_mod.quantize(synth_mod.expert_weights(8, 0, e, m, n, kk), G)
+            codes.append(cc)
+            scales.append(s)
+        experts[e] = oracle_mod.Expert(codes, scales, [cb] * 3)
+    ids = np.array([[4, 1, 3]], np.int32)
+    depth = np.array([[2, 5, 1]], np.uint8)
+    x = 3.0 * synth_mod.activation_f32(8, 0, 0, H).astype(np.float64)[None, :]
+    w = np.array([[0.5, 0.3, 0.2]], np.float32)
+    y = oracle_mod.moe_layer(experts, E, H, I, G, ids, w, depth, x)[0]
+    parts = [oracle_mod.moe_layer(experts, E, H, I, G, ids, np.eye(k, dtype=np.float32)[i:i + 1], depth, x)[0]
+             for i in range(k)]
+    np.testing.assert_allclose(y, sum(float(w[0, i]) * parts[i] for i in range(k)), rtol=1e-12, atol=1e-14)
+    y2 = oracle_mod.moe_layer(experts, E, H, I, G, ids, 2 * w, depth, x)[0]
+    np.testing.assert_allclose(y2, 2 * y, rtol=1e-12, atol=1e-14)
+    # the expert itself is not linear in x (SwiGLU): doubling x does not double y
+    y3 = oracle_mod.moe_layer(experts, E, H, I, G, ids, w, depth, 2 * x)[0]
+    assert np.linalg.norm(y3 - 2 * y) > 0.05 * np.linalg.norm(2 * y)
