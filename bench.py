@@ -197,6 +197,20 @@ def oracle_token(sens, experts, logits, x64):
     return oracle.moe_layer(need, E, H, I, G, ids, w, dep, x64)
 
 
+def host_cpu():
+    """The host's logical CPU count (nproc) and CPU model, as the baseline's context."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
+
+
 def cpu_baseline(seed):
     """The oracle, as it stands, on one full token of the workload (single thread)."""
     sens, experts, toks = oracle_token_setup(seed, [0])
@@ -208,7 +222,7 @@ def cpu_baseline(seed):
         if time.perf_counter() - t0 > 8.0 or n >= 8:
             break
     dt = time.perf_counter() - t0
-    return {"value": n / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+    return {"value": n / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle", **host_cpu(),
             "sample": f"{n} x one full batch-1 token (route, select, 10 experts x gate/up/down at "
                       f"the selected depths, SwiGLU, combine) in double, experts pre-quantised"}
 
@@ -261,7 +275,7 @@ def reference_arm(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / max(args.steps, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": layer_config(1),
-            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": 1, "kind": "oracle", **host_cpu(),
                              "sample": f"per step: {rows} rows of one selected expert matrix at its "
                                        f"selected depth (dequantise-then-matvec in double); tokens "
                                        f"counted as decoded weights / {weights_per_token}"},

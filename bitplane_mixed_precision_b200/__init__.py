@@ -50,12 +50,14 @@ _SIGS = {
     "pmoe_last_cuda_error": ([], i32),
     "pmoe_version": ([], i32),
     "pmoe_tree_codebook": ([P], i32),
+    "pmoe_tree_codebook_from_leaves": ([P, P, P], i32),
     "pmoe_quantize": ([P, i32, i32, i32, P, P, P], i32),
     "pmoe_pack_bitplanes": ([P, i32, i32, i32, P, i64, i32, P], i32),
     "pmoe_extract_prefix": ([P, i64, i32, i32, i32, P, P], i32),
     "pmoe_route": ([P, i32, i32, i32, P, P, P], i32),
     "pmoe_select_prefix": ([P, P, P, i32, i32, f32, P, i32, P], i32),
     "pmoe_select_prefix_cache_aware": ([P, P, P, P, i32, i32, i32, P], i32),
+    "pmoe_select_prefix_cache_aware_matched": ([P, P, P, P, i32, i32, f32, P, P], i32),
     "pmoe_relative_error": ([P, P, i32, i32, P, P], i32),
     "pmoe_profile_repair": ([P, i32, P], i32),
     "pmoe_select_prefix_table": ([P, P, P, i32, i32, f32, P, i32, P], i32),
@@ -73,6 +75,7 @@ _SIGS = {
     "pmoe_cache_create": ([i32, i32, i64, i64, P, P, i32, ctypes.POINTER(P)], i32),
     "pmoe_cache_extend": ([P, i32, P, P, i32, i64, P, P, P, P, P, ctypes.POINTER(CacheStats)], i32),
     "pmoe_cache_get_stats": ([P, ctypes.POINTER(CacheStats)], i32),
+    "pmoe_cache_inject_copy_failure": ([P, i64], i32),
     "pmoe_cache_resident_depth": ([P, i32, P], i32),
     "pmoe_cache_eviction_log": ([P, P, i64, ctypes.POINTER(i64)], i32),
     "pmoe_cache_destroy": ([P], i32),
@@ -135,6 +138,12 @@ def tree_codebook(out) -> None:
     _check("pmoe_tree_codebook", _lib.pmoe_tree_codebook(_ptr(out)))
 
 
+def tree_codebook_from_leaves(leaves, freq, out) -> None:
+    """Host float32 arrays: 256 sorted leaves, 256 frequencies -> 510-entry tree."""
+    _check("pmoe_tree_codebook_from_leaves", _lib.pmoe_tree_codebook_from_leaves(_ptr(leaves), _ptr(freq),
+                                                                               _ptr(out)))
+
+
 def quantize(w, N, K, G, scales, codes, stream=None) -> None:
     _check("pmoe_quantize", _lib.pmoe_quantize(_ptr(w), N, K, G, _ptr(scales), _ptr(codes), _stream(stream)))
 
@@ -163,6 +172,13 @@ def select_prefix_cache_aware(w, ids, sens, resident, T, k, fetch_budget, depth)
     """Host arrays; depths under a budget of fetched planes per token (resident planes free)."""
     _check("pmoe_select_prefix_cache_aware", _lib.pmoe_select_prefix_cache_aware(
         _ptr(w), _ptr(ids), _ptr(sens), _ptr(resident), T, k, int(fetch_budget), _ptr(depth)))
+
+
+def select_prefix_cache_aware_matched(w, ids, sens, resident, T, k, avg_bits, depth, surrogate=None) -> None:
+    """Host arrays; the cache-aware depths with the cache-oblivious depths' fetch count as budget.
+    surrogate: optional float64 numpy [2] accumulating sum (w s)^2 4^-b (oblivious, returned)."""
+    _check("pmoe_select_prefix_cache_aware_matched", _lib.pmoe_select_prefix_cache_aware_matched(
+        _ptr(w), _ptr(ids), _ptr(sens), _ptr(resident), T, k, avg_bits, _ptr(depth), _ptr(surrogate)))
 
 
 def relative_error(y, ref, T, H, err, stream=None) -> None:
@@ -289,6 +305,10 @@ class Cache:
             self._h, layer, _ptr(experts), _ptr(need), len(experts), int(batch), self._host_ptrs,
             _stream(side), _event(after), _event(done), _ptr(resident_before), ctypes.byref(st)))
         return st
+
+    def inject_copy_failure(self, nth):
+        """Testing hook: the nth next plane copy reports failure (0 disarms)."""
+        _check("pmoe_cache_inject_copy_failure", _lib.pmoe_cache_inject_copy_failure(self._h, int(nth)))
 
     def stats(self):
         st = CacheStats()

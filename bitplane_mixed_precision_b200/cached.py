@@ -24,7 +24,7 @@ import numpy as np
 import torch
 
 from . import Cache, make_layer, moe_layer_fwd, layer_workspace_bytes, residual_norm, route_host, \
-    select_prefix, select_prefix_cache_aware, layer_error
+    select_prefix_cache_aware_matched, layer_error
 
 
 class CachedStack:
@@ -66,7 +66,7 @@ class CachedStack:
         # depths would fetch are the budget, and resident planes come free
         self.cache_aware = cache_aware
         self.keep_log = keep_log
-        self.surrogate = [0.0, 0.0]  # sum of w^2 s^2 4^-b: cache-oblivious depths, depths used
+        self._sur = np.zeros(2, np.float64)  # sum of (w s)^2 4^-b: cache-oblivious depths, depths used
         self.side = torch.cuda.Stream(dev)
         self.done = [torch.cuda.Event() for _ in range(L)]
         for e in self.done:  # torch creates the CUDA event at its first record; the library records it
@@ -89,16 +89,15 @@ class CachedStack:
         self.trace = []
 
     def _select(self, l, ids, w, dep):
-        """Depths of layer l's slots (host arrays of one token); cache-aware when enabled."""
+        """Depths of layer l's slots (host arrays of one token). Cache-aware: resident planes are
+        free and the budget is what the cache-oblivious depths would fetch. Otherwise the same
+        call with nothing counted as resident, which is the plain allocator."""
         sens = self.sens[l % len(self.sens)]
-        select_prefix(w, ids, sens, 1, self.k, self.avg_bits, dep, on_device=False)
-        v2 = (w.astype(np.float64) * sens[ids].astype(np.float64)) ** 2
-        self.surrogate[0] += float(np.sum(v2 * 4.0 ** (-dep.astype(np.float64))))
         if self.cache_aware:
-            res = self.cache.resident_depth(l)[ids].astype(np.uint8)
-            fetch = int(np.maximum(dep.astype(np.int64) - res, 0).sum())
-            select_prefix_cache_aware(w, ids, sens, res, 1, self.k, fetch, dep)
-        self.surrogate[1] += float(np.sum(v2 * 4.0 ** (-dep.astype(np.float64))))
+            res = np.ascontiguousarray(self.cache.resident_depth(l)[ids], dtype=np.uint8)
+        else:
+            res = np.zeros(self.k, np.uint8)
+        select_prefix_cache_aware_matched(w, ids, sens, res, 1, self.k, self.avg_bits, dep, self._sur)
 
     def plan(self, logits, t):
         """Host routing for all layers of token t (logits: float32 [L, E]); returns the set."""
@@ -150,8 +149,13 @@ class CachedStack:
         nb = len(self.host)
         self.cache.set_host_planes([self.host[l % nb] for l in range(self.L)])
         self.trace = []
-        self.surrogate = [0.0, 0.0]
+        self._sur[:] = 0.0
         self.token_done_valid = False
+
+    @property
+    def surrogate(self):
+        """[sum of (w s)^2 4^-b with the cache-oblivious depths, with the depths used]."""
+        return [float(self._sur[0]), float(self._sur[1])]
 
     def routing(self, s):
         """Host copies (ids, w, depth) of the token planned into set s."""

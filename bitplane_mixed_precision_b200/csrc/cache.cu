@@ -75,6 +75,7 @@ struct pmoe_cache {
     int64_t clock = 0;
     pmoe_cache_stats stats{};
     std::vector<int64_t> log;
+    int64_t fail_copy_in = 0; // > 0: the fail_copy_in-th next host-to-device copy reports failure (testing)
 
     // page-table updates staged in mapped pinned memory
     int2 *stage = nullptr;
@@ -214,18 +215,27 @@ pmoe_status pmoe_cache_extend(pmoe_cache *c, int layer, const int32_t *experts, 
             touched.push_back((int)k);
         }
     };
-    struct Copy {
-        int32_t slot;
-        int64_t from; // word offset in the layer's host planes
-    };
-    std::vector<Copy> copies;
-    bool evicted = false;
+    bool waited_after = false; // `side` waits for `after` before the first copy into an evicted slot
     pmoe_status rc = PMOE_OK;
+    // Enqueues one plane copy; the testing hook can make it report failure without enqueueing.
+    auto copy_plane = [&](int32_t slot, int64_t from) -> pmoe_status {
+        if (c->fail_copy_in > 0 && --c->fail_copy_in == 0) {
+            set_cuda_error(cudaErrorInvalidValue);
+            return PMOE_ERR_CUDA;
+        }
+        return cuda_status(cudaMemcpyAsync(c->pool + (int64_t)slot * c->slot_words, src + from,
+                                           (size_t)c->slot_words * 4, cudaMemcpyHostToDevice, st));
+    };
 
     for (int i = 0; i < n; ++i) {
         const int e = experts[i], b = need[i];
         const int64_t x = (int64_t)layer * c->E + e;
         const int r = c->depth[(size_t)x];
+        // what this access changes on the entry, so that a failed copy can take it back
+        int64_t old_ts[8];
+        for (int p = 0; p < 8; ++p)
+            old_ts[p] = c->ts[(size_t)x * 8 + p];
+        const int64_t old_batch = c->last_batch[(size_t)x];
         const int64_t now = c->clock++;
         if (resident_before)
             resident_before[i] = (uint8_t)r;
@@ -243,6 +253,7 @@ pmoe_status pmoe_cache_extend(pmoe_cache *c, int layer, const int32_t *experts, 
         for (int p = 0; p < r; ++p)
             c->ts[(size_t)x * 8 + p] = now;
         const int want = b - r;
+        bool evicted_here = false;
         // evict the oldest deepest planes of entries outside this batch until the suffix fits
         while (c->used + want > c->slots) {
             auto it = c->order.begin();
@@ -265,22 +276,48 @@ pmoe_status pmoe_cache_extend(pmoe_cache *c, int layer, const int32_t *experts, 
                 c->log.push_back(y * 8 + p);
             if (c->depth[(size_t)y] > 0)
                 c->order.insert({c->deepest_ts(y), y});
-            evicted = true;
+            evicted_here = true;
         }
         if (rc != PMOE_OK) {
             if (r > 0)
                 c->order.insert({c->deepest_ts(x), x});
             break;
         }
-        for (int p = r; p < b; ++p) {
-            const int32_t s = c->free_slots.back();
+        if (moves && evicted_here && after && !waited_after) {
+            rc = cuda_status(cudaStreamWaitEvent(st, (cudaEvent_t)after, 0));
+            waited_after = rc == PMOE_OK;
+        }
+        int p_ok = r; // planes r..p_ok-1 have their copies enqueued
+        for (int p = r; p < b && rc == PMOE_OK; ++p) {
+            const int32_t slot = c->free_slots.back();
+            if (moves)
+                rc = copy_plane(slot, ((int64_t)e * 8 + p) * c->slot_words);
+            if (rc != PMOE_OK)
+                break;
             c->free_slots.pop_back();
             const size_t k = (size_t)x * 8 + p;
-            c->pt[k] = s;
+            c->pt[k] = slot;
             c->ts[k] = now;
             touch(k);
-            if (moves)
-                copies.push_back({s, ((int64_t)e * 8 + p) * c->slot_words});
+            p_ok = p + 1;
+        }
+        if (rc != PMOE_OK) {
+            // a copy could not be enqueued: this access is taken back. Its planes whose copies were
+            // enqueued go back to the free list (their data lands in free slots); the entry keeps
+            // its depth, times and batch as before the access; the evictions above stay (the
+            // enqueued copies may have overwritten evicted slots).
+            for (int p = p_ok - 1; p >= r; --p) {
+                const size_t k = (size_t)x * 8 + p;
+                c->free_slots.push_back(c->pt[k]);
+                c->pt[k] = -1;
+            }
+            for (int p = 0; p < 8; ++p)
+                c->ts[(size_t)x * 8 + p] = old_ts[p];
+            c->last_batch[(size_t)x] = old_batch;
+            c->stats.requests -= 1;
+            if (r > 0)
+                c->order.insert({c->deepest_ts(x), x});
+            break;
         }
         c->depth[(size_t)x] = (uint8_t)b;
         c->used += want;
@@ -289,26 +326,35 @@ pmoe_status pmoe_cache_extend(pmoe_cache *c, int layer, const int32_t *experts, 
         c->order.insert({c->deepest_ts(x), x});
     }
 
-    // an entry evicted and fetched again in one call is written once, with its final slot
+    // the device page table follows the host state, also after an error: entries changed by
+    // this call are written once, with their final value
     std::vector<int2> upd;
     upd.reserve(touched.size());
     for (int k : touched) {
         upd.push_back(make_int2(k, c->pt[(size_t)k]));
         c->dirty[(size_t)k] = 0;
     }
-    if (moves && (!copies.empty() || !upd.empty())) {
-        if (evicted && after)
-            PMOE_CUDA(cudaStreamWaitEvent(st, (cudaEvent_t)after, 0));
-        for (const Copy &cp : copies)
-            PMOE_CUDA(cudaMemcpyAsync(c->pool + (int64_t)cp.slot * c->slot_words, src + cp.from,
-                                      (size_t)c->slot_words * 4, cudaMemcpyHostToDevice, st));
-        PMOE_TRY(flush_updates(c, upd, st));
+    if (moves && !upd.empty()) {
+        const pmoe_status f = flush_updates(c, upd, st);
+        if (rc == PMOE_OK)
+            rc = f;
     }
-    if (moves && done)
-        PMOE_CUDA(cudaEventRecord((cudaEvent_t)done, st));
+    if (moves && done) {
+        const pmoe_status f = cuda_status(cudaEventRecord((cudaEvent_t)done, st));
+        if (rc == PMOE_OK)
+            rc = f;
+    }
     if (stats)
         *stats = c->stats;
     return rc;
+}
+
+pmoe_status pmoe_cache_inject_copy_failure(pmoe_cache *c, int64_t nth)
+{
+    if (!c || nth < 0)
+        return PMOE_ERR_INVALID_ARG;
+    c->fail_copy_in = nth;
+    return PMOE_OK;
 }
 
 pmoe_status pmoe_cache_get_stats(const pmoe_cache *c, pmoe_cache_stats *stats)

@@ -256,6 +256,37 @@ pmoe_status pmoe_tree_codebook(float *codebook)
     return PMOE_OK;
 }
 
+pmoe_status pmoe_tree_codebook_from_leaves(const float *leaves, const float *freq, float *codebook)
+{
+    if (!leaves || !freq || !codebook)
+        return PMOE_ERR_INVALID_ARG;
+    for (int i = 0; i < 256; ++i) {
+        if (!(freq[i] >= 0.0f) || !std::isfinite(freq[i]) || !std::isfinite(leaves[i]))
+            return PMOE_ERR_INVALID_ARG;
+        if (i > 0 && leaves[i] < leaves[i - 1])
+            return PMOE_ERR_INVALID_ARG;
+    }
+    // node values and masses of the level below, in double; depth 8 = the leaves
+    double val[256], mass[256];
+    for (int i = 0; i < 256; ++i) {
+        val[i] = (double)leaves[i];
+        mass[i] = (double)freq[i];
+        codebook[254 + i] = leaves[i];
+    }
+    for (int d = 7; d >= 1; --d) {
+        const int n = 1 << d;
+        for (int i = 0; i < n; ++i) {
+            const double m0 = mass[2 * i], m1 = mass[2 * i + 1];
+            const double v = (m0 + m1 > 0.0) ? (m0 * val[2 * i] + m1 * val[2 * i + 1]) / (m0 + m1)
+                                             : 0.5 * (val[2 * i] + val[2 * i + 1]);
+            val[i] = v;
+            mass[i] = m0 + m1;
+            codebook[n - 2 + i] = (float)v;
+        }
+    }
+    return PMOE_OK;
+}
+
 pmoe_status pmoe_quantize(const float *w, int N, int K, int G, float *scales, uint8_t *codes,
                           pmoe_stream stream)
 {

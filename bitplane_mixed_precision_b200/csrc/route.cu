@@ -1,5 +1,6 @@
 // Routing (top-k + softmax, PagedMoE transcript cue 4) and prefix selection
 // (greedy bit allocation on w^2 * E_e(b), transcript cues 29-31).
+#include <cmath>
 #include "common.h"
 #include "dev.cuh"
 #include "route.cuh"
@@ -133,6 +134,34 @@ pmoe_status pmoe_select_prefix_cache_aware(const float *w, const int32_t *ids, c
         }
         for (int i = 0; i < k; ++i)
             depth[t * k + i] = (uint8_t)b[i];
+    }
+    return PMOE_OK;
+}
+
+pmoe_status pmoe_select_prefix_cache_aware_matched(const float *w, const int32_t *ids, const float *sens,
+                                                   const uint8_t *resident, int T, int k, float avg_bits,
+                                                   uint8_t *depth, double *surrogate)
+{
+    if (!w || !ids || !sens || !resident || !depth || T < 0 || k < 1 || k > 32 || !(avg_bits == avg_bits))
+        return PMOE_ERR_INVALID_ARG;
+    for (int t = 0; t < T; ++t) {
+        const float *wt = w + (int64_t)t * k;
+        const int32_t *it = ids + (int64_t)t * k;
+        const uint8_t *rt = resident + (int64_t)t * k;
+        uint8_t plain[32];
+        select_host(wt, it, sens, 1, k, avg_bits, plain);
+        // the budget: planes the cache-oblivious depths would fetch for this token
+        int fetch = 0;
+        for (int i = 0; i < k; ++i)
+            fetch += plain[i] > rt[i] ? plain[i] - rt[i] : 0;
+        PMOE_TRY(pmoe_select_prefix_cache_aware(wt, it, sens, rt, 1, k, fetch, depth + (int64_t)t * k));
+        if (surrogate) {
+            for (int i = 0; i < k; ++i) {
+                const double v = (double)wt[i] * (double)sens[it[i]];
+                surrogate[0] += v * v * std::ldexp(1.0, -2 * plain[i]);
+                surrogate[1] += v * v * std::ldexp(1.0, -2 * depth[(int64_t)t * k + i]);
+            }
+        }
     }
     return PMOE_OK;
 }

@@ -89,6 +89,20 @@ PMOE_API int pmoe_version(void);
 PMOE_API pmoe_status pmoe_tree_codebook(float *codebook);
 
 /*
+ * pmoe_tree_codebook_from_leaves [T#19, T#21]: the tree codebook of a sorted
+ * 256-entry leaf table (for example a per-block K-means codebook): the leaves
+ * are depth 8, and every parent is the frequency-weighted mean of its two
+ * children, carrying the sum of their frequencies (a pair with both
+ * frequencies zero gets the plain mean). Computed in double level by level,
+ * stored as float. Host only, synchronous.
+ *   leaves: host float[256], ascending. freq: host float[256], >= 0 (e.g. how
+ *   many weights each leaf quantises). codebook: host float[510], written.
+ *   Returns PMOE_ERR_INVALID_ARG for NULL, unsorted leaves, a negative or
+ *   non-finite value.
+ */
+PMOE_API pmoe_status pmoe_tree_codebook_from_leaves(const float *leaves, const float *freq, float *codebook);
+
+/*
  * pmoe_quantize: per-group scale and 8-bit index of every weight for the
  * Gaussian tree codebook. scale = population std (double, sequential sum,
  * rounded to float; 0 -> 1) of the G weights of a row group; index = number
@@ -161,6 +175,23 @@ PMOE_API pmoe_status pmoe_select_prefix_cache_aware(const float *w, const int32_
                                                     uint8_t *depth);
 
 /*
+ * pmoe_select_prefix_cache_aware_matched [T#29, T#61]: the cache-aware
+ * allocator with its budget matched to the cache-oblivious one, per token:
+ * the depths pmoe_select_prefix(avg_bits) would pick determine the planes
+ * they would fetch given resident[], and that count is the fetch budget of
+ * pmoe_select_prefix_cache_aware, whose depths are returned. Both choices
+ * therefore move the same bytes; resident planes come free.
+ *   Host pointers, synchronous; arguments as pmoe_select_prefix_cache_aware.
+ *   surrogate: NULL, or host double[2] to which the call adds the error
+ *   surrogate sum of (w*s_e)^2 * 4^-b over its slots, [0] for the
+ *   cache-oblivious depths and [1] for the returned ones (w*s_e in double).
+ */
+PMOE_API pmoe_status pmoe_select_prefix_cache_aware_matched(const float *w, const int32_t *ids, const float *sens,
+                                                            const uint8_t *resident, int T, int k, float avg_bits,
+                                                            uint8_t *depth, double *surrogate);
+
+/*
+ * Profile-driven allocation [T#29, T#31]./*
  * Profile-driven allocation [T#29, T#31]. An expert's error profile E_e(b),
  * b = 1..8, is its relative output error at depth b, measured offline on
  * random Gaussian inputs; the allocator then grants bits by the profile's
@@ -386,12 +417,27 @@ PMOE_API pmoe_status pmoe_cache_create(int layers, int experts, int64_t slots, i
  *   NULL). Host-only caches ignore host_planes, side, after and done.
  * Errors: PMOE_ERR_INVALID_ARG (nothing changed); PMOE_ERR_OUT_OF_SLOTS
  * when the pinned entries of the batch leave no room (the accesses before
- * the failing one are applied and their copies enqueued); PMOE_ERR_CUDA.
+ * the failing one are applied and their copies enqueued); PMOE_ERR_CUDA when
+ * a copy, the page-table kernel or an event call cannot be enqueued. For a
+ * copy that cannot be enqueued, the accesses before it are applied; its own
+ * access is taken back (depth, plane times, batch and counters as before
+ * it; slots it took are free again) and later accesses are not made; planes
+ * evicted on its behalf stay evicted, since copies already enqueued may
+ * overwrite their slots. In every case the device page table is brought in
+ * line with the host state before the call returns.
  */
 PMOE_API pmoe_status pmoe_cache_extend(pmoe_cache *c, int layer, const int32_t *experts, const uint8_t *need,
                                        int n, int64_t batch, const uint32_t *const *host_planes,
                                        pmoe_stream side, pmoe_event after, pmoe_event done,
                                        uint8_t *resident_before, pmoe_cache_stats *stats);
+
+/*
+ * pmoe_cache_inject_copy_failure (testing hook): the nth next host-to-device
+ * plane copy of this cache (nth >= 1) reports failure instead of being
+ * enqueued, as a failing cudaMemcpyAsync would (PMOE_ERR_CUDA, last CUDA error
+ * cudaErrorInvalidValue); nth = 0 disarms. Host state only; touches no GPU.
+ */
+PMOE_API pmoe_status pmoe_cache_inject_copy_failure(pmoe_cache *c, int64_t nth);
 
 /* Accumulated counters. */
 PMOE_API pmoe_status pmoe_cache_get_stats(const pmoe_cache *c, pmoe_cache_stats *stats);

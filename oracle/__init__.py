@@ -43,6 +43,7 @@ def _l():
             "or_norm_ppf": ([f64], f64),
             "or_tree_codebook": ([P], None),
             "or_tree_codebook_f32": ([P], None),
+            "or_tree_from_leaves": ([P, P, P], None),
             "or_thresholds": ([P], None),
             "or_quantize": ([P, i32, i32, i32, P, P], None),
             "or_pack": ([P, i32, i32, i32, P], i32),
@@ -88,6 +89,16 @@ def tree_codebook() -> np.ndarray:
 def tree_codebook_f32() -> np.ndarray:
     out = np.empty(510, dtype=np.float32)
     _l().or_tree_codebook_f32(_p(out))
+    return out
+
+
+def tree_from_leaves(leaves, freq) -> np.ndarray:
+    """510 doubles: the tree over 256 sorted leaves, parents the frequency-weighted means."""
+    leaves = np.ascontiguousarray(leaves, dtype=np.float64)
+    freq = np.ascontiguousarray(freq, dtype=np.float64)
+    assert leaves.shape == (256,) and freq.shape == (256,)
+    out = np.empty(510, dtype=np.float64)
+    _l().or_tree_from_leaves(_p(leaves), _p(freq), _p(out))
     return out
 
 

@@ -96,6 +96,39 @@ void or_tree_codebook_f32(float *cb /* [510] */)
         cb[i] = (float)tmp[i];
 }
 
+/*
+ * Tree codebook from a sorted 256-entry leaf set with leaf frequencies
+ * [T#19, T#21]: the leaves sit at depth 8 in sorted order; every parent is
+ * the frequency-weighted mean of its two children and carries the sum of
+ * their frequencies, level by level up to depth 1. A pair whose frequencies
+ * are both zero gets the plain mean of its children (and frequency 0).
+ * Storage as or_tree_codebook. All in double.
+ * Pins: equal frequencies on the Gaussian leaves give the closed-form tree
+ * (equal-mass children); every node equals the weighted average of the leaves
+ * below it (numpy, computed directly from the leaves, not level by level).
+ */
+void or_tree_from_leaves(const double *leaves /* [256] */, const double *freq /* [256] */,
+                         double *cb /* [510] */)
+{
+    double f[256], v[256];
+    for (int i = 0; i < 256; ++i) {
+        v[i] = leaves[i];
+        f[i] = freq[i];
+        cb[254 + i] = leaves[i];
+    }
+    for (int d = 7; d >= 1; --d) {
+        int n = 1 << d;
+        for (int i = 0; i < n; ++i) {
+            double fl = f[2 * i], fr = f[2 * i + 1];
+            double m = (fl + fr > 0.0) ? (fl * v[2 * i] + fr * v[2 * i + 1]) / (fl + fr)
+                                       : 0.5 * (v[2 * i] + v[2 * i + 1]);
+            v[i] = m;
+            f[i] = fl + fr;
+            cb[(n - 2) + i] = m;
+        }
+    }
+}
+
 /* ------------------------------------------------------------------ */
 /* Quantiser: per-group std scale, 256 equiprobable N(0,1) bins         */
 /* ------------------------------------------------------------------ */

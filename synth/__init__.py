@@ -34,7 +34,7 @@ _HOST_SO = os.path.join(_HERE, "libpmoe_synth.so")
 _DEV_SO = os.path.join(_HERE, "libpmoe_synth_dev.so")
 
 # stream kinds
-K_WEIGHT, K_X, K_LOGIT, K_SENS, K_PERM, K_AR = 1, 2, 3, 4, 5, 6
+K_WEIGHT, K_X, K_LOGIT, K_SENS, K_PERM, K_AR, K_LEAF = 1, 2, 3, 4, 5, 6, 7
 
 
 def build(force: bool = False, device: bool = True) -> None:
@@ -188,6 +188,23 @@ def ar1_logits(seed: int, layer: int, tokens: int, experts: int, rho: float = 0.
     for t in range(1, tokens):
         out[t] = rho * out[t - 1] + c * e[t]
     return out.astype(np.float32)
+
+
+def tree_leaves(seed: int, table: int = 0):
+    """A skewed, heavy-tailed 256-entry leaf table, ascending, and leaf frequencies (float32).
+
+    Stands in for a per-block K-means codebook of real weights: draws
+    t = z0 / sqrt((z1^2 + z2^2 + z3^2) / 3) (Student-t, 3 degrees of freedom)
+    plus a skew term 0.4 * |z0|, sorted; frequencies 1 + 999 * u with u
+    uniform in [0, 1) from the counter stream, and two of them set to zero."""
+    z = normal_f64(seed, stream_id(K_LEAF, table), 4 * 256).reshape(4, 256)
+    t = z[0] / np.sqrt((z[1] ** 2 + z[2] ** 2 + z[3] ** 2) / 3.0) + 0.4 * np.abs(z[0])
+    leaves = np.sort(t).astype(np.float32)
+    u = u64(seed, stream_id(K_LEAF, table, 1), 256)
+    freq = (1.0 + 999.0 * (u >> np.uint64(11)).astype(np.float64) / float(1 << 53)).astype(np.float32)
+    freq[7] = 0.0
+    freq[8] = 0.0
+    return leaves, freq
 
 
 @dataclass

@@ -120,3 +120,35 @@ def test_profile_repair_and_table_select_match_oracle(pm, oracle_mod):
     got = np.zeros((T, k), np.uint8)
     pm.select_prefix_table(w, ids, table, T, k, 2.5, got, on_device=False)
     assert np.array_equal(got, oracle_mod.select_table(w, ids, table, 2.5))
+
+
+def test_cache_aware_matched_against_oracle():
+    """pmoe_select_prefix_cache_aware_matched = the oracle's cache-aware selection with the fetch
+    budget of the oracle's plain depths, and its surrogate sums; with nothing resident it is the
+    plain allocator."""
+    import oracle
+    import synth
+    import bitplane_mixed_precision_b200 as pm
+    E, k, T = 512, 10, 64
+    sens = synth.sensitivities(77, 0, E)
+    logits = np.stack([synth.router_logits(77, t, 0, E) for t in range(T)])
+    ids, w = oracle.route(logits, k)
+    rng = np.random.default_rng(5)
+    res = rng.integers(0, 9, (T, k)).astype(np.uint8)
+    res[::3] = 0
+    dep = np.empty((T, k), np.uint8)
+    sur = np.zeros(2)
+    pm.select_prefix_cache_aware_matched(w, ids, sens, res, T, k, 2.5, dep, sur)
+    plain = oracle.select(w, ids, sens, 2.5)
+    want_sur = np.zeros(2)
+    for t in range(T):
+        fetch = int(np.maximum(plain[t].astype(int) - res[t].astype(int), 0).sum())
+        ref = oracle.select_cache_aware(w[t:t + 1], ids[t:t + 1], sens, res[t:t + 1], fetch)[0]
+        np.testing.assert_array_equal(dep[t], ref)
+        v2 = (w[t].astype(np.float64) * sens[ids[t]].astype(np.float64)) ** 2
+        want_sur += [np.sum(v2 * 4.0 ** -plain[t].astype(float)), np.sum(v2 * 4.0 ** -ref.astype(float))]
+    np.testing.assert_allclose(sur, want_sur, rtol=1e-12)
+    assert sur[1] <= sur[0]
+    zero = np.zeros((T, k), np.uint8)
+    pm.select_prefix_cache_aware_matched(w, ids, sens, zero, T, k, 2.5, dep, None)
+    np.testing.assert_array_equal(dep, plain)

@@ -184,3 +184,61 @@ def test_profile_driven_allocation(stack_setup, synth_mod, oracle_mod):
     torch.cuda.synchronize()
     assert np.array_equal(devd.cpu().numpy(), host)
     assert np.array_equal(host, oracle_mod.select_table(w, ids, table, AVG))
+
+
+def test_injected_copy_failure_takes_the_access_back(stack_setup):
+    """A plane copy that cannot be enqueued (host-side injection): the call returns PMOE_ERR_CUDA,
+    the accesses before the failing one are applied, the failing access and the rest are not,
+    and the device page table equals the host state; the cache keeps working afterwards."""
+    import bitplane_mixed_precision_b200 as pm
+    dev, backs, sens = stack_setup
+    slot_words = 3 * H * I // 32
+    slots = 40
+    pool = torch.zeros(slots * slot_words, dtype=torch.int32, device=dev)
+    pt = torch.full((L * E * 8,), -1, dtype=torch.int32, device=dev)
+    c = pm.Cache(L, E, slots, slot_words, pool, pt)
+    host = torch.empty(E * 8 * slot_words, dtype=torch.int32).pin_memory()
+    host.copy_(backs[0].pool)
+    c.set_host_planes([host] * L)
+    side = torch.cuda.Stream(dev)
+
+    def device_pt_matches():
+        torch.cuda.synchronize()
+        got = pt.cpu().numpy().reshape(L, E, 8)
+        for l in range(L):
+            d = c.resident_depth(l)
+            for e in range(E):
+                assert np.all(got[l, e, :d[e]] >= 0) and np.all(got[l, e, d[e]:] == -1), (l, e)
+
+    # the first copy fails: nothing is applied
+    c.inject_copy_failure(1)
+    with pytest.raises(pm.PmoeError) as ei:
+        c.extend(0, np.array([3, 5], np.int32), np.array([2, 1], np.uint8), 0, side=side)
+    assert ei.value.code == 2
+    st = c.stats()
+    assert (st.requests, st.hits, st.planes_fetched, st.planes_evicted) == (0, 0, 0, 0)
+    assert not c.resident_depth(0).any()
+    device_pt_matches()
+    # the fifth copy fails: expert 3 (2 planes) and expert 5 (1 plane) are applied, expert 7's
+    # access (its first plane copied, its second failing) and expert 9's are not
+    c.inject_copy_failure(5)
+    with pytest.raises(pm.PmoeError):
+        c.extend(0, np.array([3, 5, 7, 9], np.int32), np.array([2, 1, 3, 1], np.uint8), 1, side=side)
+    d = c.resident_depth(0)
+    assert (d[3], d[5], d[7], d[9]) == (2, 1, 0, 0)
+    st = c.stats()
+    assert (st.requests, st.planes_fetched) == (2, 3)
+    device_pt_matches()
+    # without injection the same request completes, and the data in the slots is the expert's
+    c.extend(0, np.array([3, 5, 7, 9], np.int32), np.array([2, 1, 3, 1], np.uint8), 2, side=side)
+    torch.cuda.synchronize()
+    d = c.resident_depth(0)
+    assert (d[3], d[5], d[7], d[9]) == (2, 1, 3, 1)
+    device_pt_matches()
+    ptn = pt.cpu().numpy().reshape(L, E, 8)
+    for e, b in ((3, 2), (5, 1), (7, 3), (9, 1)):
+        for p in range(b):
+            s = int(ptn[0, e, p])
+            want = backs[0].pool[(e * 8 + p) * slot_words:(e * 8 + p + 1) * slot_words]
+            assert torch.equal(pool[s * slot_words:(s + 1) * slot_words], want), (e, p)
+    c.close()

@@ -86,3 +86,62 @@ def test_golden_truncation_example(oracle_mod):
         c1 = oracle_mod.level(cb, 1)
         p = int(parent)
         assert c1[p] == pytest.approx(0.5 * (c2[2 * p] + c2[2 * p + 1]), abs=1e-14)
+
+
+# Tree from sorted leaves with frequencies (transcript cues 19, 21): every parent is the
+# frequency-weighted mean of its children.
+
+def test_tree_from_leaves_equal_mass_is_the_gaussian_tree(oracle_mod):
+    """Equal leaf frequencies on the Gaussian conditional-mean leaves: each parent is the plain
+    mean of its children, which is the closed-form conditional mean of the merged bin."""
+    cb = oracle_mod.tree_codebook()
+    t = oracle_mod.tree_from_leaves(oracle_mod.level(cb, 8), np.ones(256))
+    np.testing.assert_allclose(t, cb, rtol=0, atol=1e-13)
+
+
+def test_tree_from_leaves_nodes_are_subtree_weighted_averages(oracle_mod, synth_mod):
+    """Every depth-d node equals the frequency-weighted average of the 2^(8-d) leaves below it,
+    computed directly from the leaves (numpy's weighted average), not level by level."""
+    leaves, freq = synth_mod.tree_leaves(5)
+    freq = freq.astype(np.float64)
+    t = oracle_mod.tree_from_leaves(leaves, freq)
+    for d in range(1, 9):
+        lv = oracle_mod.level(t, d)
+        span = 1 << (8 - d)
+        for i in range(1 << d):
+            sl = slice(i * span, (i + 1) * span)
+            if freq[sl].sum() > 0:
+                want = np.average(leaves[sl].astype(np.float64), weights=freq[sl])
+                assert lv[i] == pytest.approx(want, rel=1e-13, abs=1e-14)
+    # leaves 7 and 8 have zero frequency: the depth-7 node above leaves 6, 7 is leaf 6, the one
+    # above 8, 9 is leaf 9
+    assert oracle_mod.level(t, 7)[3] == pytest.approx(float(leaves[6]), rel=1e-15)
+    assert oracle_mod.level(t, 7)[4] == pytest.approx(float(leaves[9]), rel=1e-15)
+
+
+def test_tree_from_leaves_zero_mass_pair_is_plain_mean(oracle_mod):
+    leaves = np.linspace(-2.0, 2.0, 256)
+    freq = np.ones(256)
+    freq[10] = freq[11] = 0.0
+    t = oracle_mod.tree_from_leaves(leaves, freq)
+    assert oracle_mod.level(t, 7)[5] == pytest.approx(0.5 * (leaves[10] + leaves[11]), rel=1e-15)
+    # its parent weighs it by zero mass: the parent is its sibling pair's mean
+    assert oracle_mod.level(t, 6)[2] == pytest.approx(0.5 * (leaves[8] + leaves[9]), rel=1e-15)
+
+
+def test_library_tree_from_leaves_equals_oracle(oracle_mod, synth_mod):
+    """The library's host builder (float output) against the oracle rounded to float."""
+    import bitplane_mixed_precision_b200 as pm
+    for seed in (1, 2, 3):
+        leaves, freq = synth_mod.tree_leaves(seed)
+        out = np.empty(510, np.float32)
+        pm.tree_codebook_from_leaves(leaves, freq, out)
+        ref = oracle_mod.tree_from_leaves(leaves, freq.astype(np.float64)).astype(np.float32)
+        np.testing.assert_array_equal(out, ref)
+    bad = np.empty(510, np.float32)
+    with pytest.raises(pm.PmoeError):
+        pm.tree_codebook_from_leaves(np.linspace(1, -1, 256).astype(np.float32), np.ones(256, np.float32), bad)
+    with pytest.raises(pm.PmoeError):
+        fr = np.ones(256, np.float32)
+        fr[3] = -1
+        pm.tree_codebook_from_leaves(np.linspace(-1, 1, 256).astype(np.float32), fr, bad)
