@@ -68,8 +68,10 @@ _SIGS = {
                              i32),
     "pmoe_profile_events": ([P, P], i32),
     "pmoe_noalloc_scratch_bytes": ([], sz),
+    "pmoe_noalloc_layer_error": ([ctypes.POINTER(i32), ctypes.POINTER(i32), P], i32),
     "pmoe_moe_layer_fwd_noalloc": ([ctypes.POINTER(Layer), P, P, P, P, i32, i32, P, P], i32),
     "pmoe_layer_error": ([P, ctypes.POINTER(i32), ctypes.POINTER(i32), P], i32),
+    "pmoe_set_wait_limit_ns": ([ctypes.c_uint64], i32),
     "pmoe_materialise_workspace_bytes": ([i32, i32, i32, i32, i32], sz),
     "pmoe_materialise_layer_fwd": ([ctypes.POINTER(Layer), P, P, P, P, i32, i32, P, P, sz, P], i32),
     "pmoe_cache_create": ([i32, i32, i64, i64, P, P, i32, ctypes.POINTER(P)], i32),
@@ -221,6 +223,14 @@ def noalloc_scratch_bytes() -> int:
     return _lib.pmoe_noalloc_scratch_bytes()
 
 
+def noalloc_layer_error(stream=None):
+    """(code, detail) of the error record in the allocation-free call's array (synchronises)."""
+    code, detail = i32(0), i32(0)
+    _check("pmoe_noalloc_layer_error", _lib.pmoe_noalloc_layer_error(ctypes.byref(code), ctypes.byref(detail),
+                                                                     _stream(stream)))
+    return code.value, detail.value
+
+
 def moe_layer_fwd_noalloc(L: Layer, x, ids, w, depth, T, k, y, stream=None) -> None:
     """pmoe_moe_layer_fwd with the library's fixed scratch array instead of a workspace."""
     _check("pmoe_moe_layer_fwd_noalloc", _lib.pmoe_moe_layer_fwd_noalloc(
@@ -241,6 +251,11 @@ def profile_events(start, stop) -> None:
             return None
         return e.cuda_event if hasattr(e, "cuda_event") else int(e)
     _check("pmoe_profile_events", _lib.pmoe_profile_events(h(start), h(stop)))
+
+
+def set_wait_limit_ns(ns) -> None:
+    """Bound of the layer kernels' device waits (0 = the default, 200 ms)."""
+    _check("pmoe_set_wait_limit_ns", _lib.pmoe_set_wait_limit_ns(int(ns)))
 
 
 def layer_error(ws, stream=None):

@@ -60,6 +60,13 @@ LayerWs carve_layer_ws(void *ws, int T, int k, int H, int I, size_t *bytes)
     const size_t o_hf = take(P * (I / 32) * 16 * 4), o_he = take(P * (size_t)hexp_stride(I) * 4);
     const size_t o_part = take(P * H * 4);
     const size_t o_ids = take(P * 4), o_w = take(P * 4), o_dep = take(P);
+    // batch-1 kernel only
+    const size_t P1 = (T == 1) ? (size_t)k : 0;
+    const size_t nka = (size_t)H / 256, nkb = 8;
+    const size_t o_pa1 = take(P1 * (I / 16) * nka * 32 * 4), o_pea = take(P1 * (I / 16) * nka * 4);
+    const size_t o_pb1 = take(P1 * (H / 16) * nkb * 16 * 4), o_peb = take(P1 * (H / 16) * nkb * 4);
+    const size_t o_cb1 = take(P1 * (H / 16) * 4), o_rh = take(P1 * (I / 128) * 4);
+    const size_t o_yc1 = take(T == 1 ? (size_t)(H / 16) * 4 : 0);
     if (bytes)
         *bytes = off;
     LayerWs L{};
@@ -90,6 +97,13 @@ LayerWs carve_layer_ws(void *ws, int T, int k, int H, int I, size_t *bytes)
     L.hfrag = reinterpret_cast<uint32_t *>(b + o_hf);
     L.hexp = reinterpret_cast<int *>(b + o_he);
     L.part = reinterpret_cast<float *>(b + o_part);
+    L.pA1 = reinterpret_cast<float *>(b + o_pa1);
+    L.pendA = reinterpret_cast<int *>(b + o_pea);
+    L.pB1 = reinterpret_cast<float *>(b + o_pb1);
+    L.pendB = reinterpret_cast<int *>(b + o_peb);
+    L.cntB1 = reinterpret_cast<int *>(b + o_cb1);
+    L.readyH = reinterpret_cast<int *>(b + o_rh);
+    L.ycnt1 = reinterpret_cast<int *>(b + o_yc1);
     L.ids = reinterpret_cast<int32_t *>(b + o_ids);
     L.w = reinterpret_cast<float *>(b + o_w);
     L.depth = reinterpret_cast<uint8_t *>(b + o_dep);
@@ -332,6 +346,8 @@ pmoe_status launch_layer(const pmoe_layer *L, const float *logits, const float *
     if (ws_bytes < need)
         return PMOE_ERR_WORKSPACE;
     LayerWs W = carve_layer_ws(ws, T, k, L->H, L->I, nullptr);
+    if (T == 1)
+        return launch_decode1(L, logits, sens, x, ids, w, depth, k, B, y, W, st, g_prof_start, g_prof_stop);
     const int P = T * k;
     const bool frags_here = (int64_t)T * (L->H / 128) <= 128;
     if (!frags_here) {
@@ -361,7 +377,7 @@ pmoe_status launch_layer(const pmoe_layer *L, const float *logits, const float *
         return PMOE_ERR_UNSUPPORTED;
     if (g_num_sms[dev] == 0)
         PMOE_CUDA(cudaDeviceGetAttribute(&g_num_sms[dev], cudaDevAttrMultiProcessorCount, dev));
-    mk::Args ma{*L, T, k, w, y, W};
+    mk::Args ma{*L, T, k, w, y, W, wait_limit_ns()};
     const size_t smem = sizeof(mk::Smem);
     void (*kern)(mk::Args);
     switch (L->G) {
@@ -411,6 +427,12 @@ size_t pmoe_layer_workspace_bytes(int T, int k, int E, int H, int I)
     size_t b = 0;
     carve_layer_ws(nullptr, T, k, H, I, &b);
     return b;
+}
+
+pmoe_status pmoe_set_wait_limit_ns(uint64_t ns)
+{
+    set_wait_limit_ns(ns == 0 ? 200ull * 1000 * 1000 : ns);
+    return PMOE_OK;
 }
 
 pmoe_status pmoe_layer_error(const void *ws, int *code, int *detail, pmoe_stream stream)

@@ -21,7 +21,9 @@ void *g_noalloc_ptr[128] = {};
 }
 
 // Device address of the scratch array on the current device; looked up once
-// per device (the host-side symbol is only a stand-in for it).
+// per device (the host-side symbol is only a stand-in for it) and kept for the
+// life of the process, so the library is not to be used across a reset of the
+// device (cudaDeviceReset).
 static pmoe_status noalloc_scratch(void **out)
 {
     int dev = 0;
@@ -45,6 +47,22 @@ static pmoe_status noalloc_scratch(void **out)
 using namespace pmoe;
 
 extern "C" size_t pmoe_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+extern "C" pmoe_status pmoe_noalloc_layer_error(int *code, int *detail, pmoe_stream stream)
+{
+    if (!code)
+        return PMOE_ERR_INVALID_ARG;
+    void *ws = nullptr;
+    PMOE_TRY(noalloc_scratch(&ws));
+    // the error record is the first words of the array, as in a workspace (pmoe_layer_error)
+    int f[8];
+    PMOE_CUDA(cudaMemcpyAsync(f, ws, sizeof(f), cudaMemcpyDeviceToHost, (cudaStream_t)stream));
+    PMOE_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
+    *code = f[0];
+    if (detail)
+        *detail = f[4];
+    return PMOE_OK;
+}
 
 extern "C" pmoe_status pmoe_moe_layer_fwd_noalloc(const pmoe_layer *L, const uint16_t *x, const int32_t *ids,
                                                   const float *w, const uint8_t *depth, int T, int k, float *y,

@@ -84,6 +84,7 @@ struct Args {
     const float *wts; // routing weights [T*k]
     float *y;         // [T*H]
     LayerWs W;
+    uint64_t limit_ns; // bound of every wait (one deadline per launch)
 };
 
 // The units' and column blocks' layout: from the shared-memory copy when the
@@ -383,7 +384,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
     const pmoe_layer &L = a.L;
     const LayerWs &W = a.W;
     const int H = L.H, I = L.I, G = L.G, T = a.T, k = a.k;
-    const uint64_t deadline = pipe::globaltimer() + kDeadlineNs;
+    const uint64_t deadline = pipe::globaltimer() + a.limit_ns;
 
     if (tid == 0) {
         for (int s = 0; s < QDEPTH; ++s) {

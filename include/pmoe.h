@@ -298,11 +298,15 @@ PMOE_API pmoe_status pmoe_moe_layer_fwd(const pmoe_layer *L, const uint16_t *x, 
  *   Sharing: all calls on a device use the same array and it keeps the last
  *   call's contents; each call resets what must start at zero. Calls that
  *   overlap on the GPU (other streams, or without ordering between them)
- *   race on the array and give wrong results. pmoe_layer_error cannot read
- *   this array; check results instead.
+ *   race on the array and give wrong results. Errors the kernels record
+ *   there are read with pmoe_noalloc_layer_error.
+ *   The array's device address is looked up once per device and kept: do
+ *   not use the library across a reset of the device (cudaDeviceReset).
  * Arguments as pmoe_moe_layer_fwd, without ws and ws_bytes.
  */
 PMOE_API size_t pmoe_noalloc_scratch_bytes(void);
+/* pmoe_layer_error for the allocation-free call's array (synchronises the stream). */
+PMOE_API pmoe_status pmoe_noalloc_layer_error(int *code, int *detail, pmoe_stream stream);
 PMOE_API pmoe_status pmoe_moe_layer_fwd_noalloc(const pmoe_layer *L, const uint16_t *x, const int32_t *ids,
                                                 const float *w, const uint8_t *depth, int T, int k, float *y,
                                                 pmoe_stream stream);
@@ -311,9 +315,22 @@ PMOE_API pmoe_status pmoe_moe_layer_fwd_noalloc(const pmoe_layer *L, const uint1
  * pmoe_layer_error: reads the device-side error record of the last layer call
  * that used workspace ws (synchronises the stream). code: 0 none, 1 expert id
  * or depth out of range, 2 a needed plane has no slot (detail = e*8 + plane),
- * 3 a bounded wait inside the kernel ran out (detail = where).
+ * 3 a bounded wait inside the kernel ran out (detail = where), 4 a batch-1
+ * call whose routing leaves one SM more than four experts' down rows (the
+ * kernel's h staging; not reachable with k <= 32 on 148 SMs).
  */
 PMOE_API pmoe_status pmoe_layer_error(const void *ws, int *code, int *detail, pmoe_stream stream);
+
+/*
+ * pmoe_set_wait_limit_ns: bound of every wait inside the layer kernels of
+ * later pmoe_moe_layer_fwd / pmoe_moe_decode_step calls (process-wide): each
+ * launch gives up on any wait once this many nanoseconds have passed since it
+ * started, records error 3 (see pmoe_layer_error) and finishes. Waits for the
+ * kernel's own copies to land before it exits use a separate 1 s bound.
+ * 0 restores the default of 200 ms. Host only; the kernels stay correct with
+ * any limit that is not reached.
+ */
+PMOE_API pmoe_status pmoe_set_wait_limit_ns(uint64_t ns);
 
 /*
  * pmoe_moe_decode_step: the whole hot path for T tokens on the device:
