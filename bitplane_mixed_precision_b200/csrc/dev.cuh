@@ -14,9 +14,9 @@
 //    fixed point split into a high and a low signed byte.
 //  * The bytes are exactly the A operand fragments of mma.sync m16n8k32 (s8):
 //    one MMA per k-step and byte plane multiplies 16 rows x 32 columns by the
-//    activation, whose own 16-bit fixed-point value is split the same way into
-//    B columns (hi, lo) per token. Products are summed exactly in int32 per
-//    scale group, then scaled in float.
+//    activation, whose 24-bit fixed-point value is split into three bytes in
+//    B columns (high, middle, low) per token (xfrag.cuh). Products are summed
+//    exactly in int32 per scale group, then combined and scaled in float.
 // No dequantised matrix is ever written (transcript cue 37).
 #pragma once
 
@@ -85,6 +85,41 @@ __device__ __forceinline__ void split16(int v, int &hi, int &lo)
     lo = v - 256 * hi;
 }
 
+// Exponent s such that |v| * 2^s < 2^22 for every |v| <= m (m >= 0); 0 for m == 0.
+__device__ __forceinline__ int fix_exponent24(float m)
+{
+    if (!(m > 0.0f))
+        return 0;
+    int e;
+    frexpf(m, &e);
+    return 22 - e;
+}
+
+// 24-bit fixed point split: v = 65536*hi + 256*mid + lo, hi in [-64, 64], mid and lo in
+// [-128, 127] (|v| < 2^22).
+__device__ __forceinline__ void split24(int v, int &hi, int &mid, int &lo)
+{
+    const int v1 = (v + 128) >> 8;
+    lo = v - 256 * v1;
+    split16(v1, hi, mid);
+}
+
+// Products of 16-bit fixed-point weights (high byte wh, low byte wl: A operands of two MMAs)
+// and 24-bit fixed-point activations (high, middle, low byte in B columns 0, 1, 2; column 3
+// zero). Lane t = 0 holds columns (0, 1) of both MMAs, lane t = 1 columns (2, 3): with
+// dh0, dh1, dl0, dl1 the lane's int32 sums (wh by its first and second column, wl likewise),
+//   F = 256 * (256*dh0 + dh1 + dl0) + dl1,
+// and sum(w * x) = 2^8 * F(t = 0) + 2^-8 * F(t = 1), in units of the two fixed points. The
+// integer part is exact (|256*dh0 + dh1 + dl0| < 2^28 for 128 products per group).
+__device__ __forceinline__ float combine24(int dh0, int dh1, int dl0, int dl1)
+{
+    return __fmaf_rn((float)(dh0 * 256 + dh1 + dl0), 256.0f, (float)dl1);
+}
+
+// The lane factor of combine24's F: 2^8 for the lane holding columns 0, 1 of a token's three
+// byte columns, 2^-8 for the lane holding its columns 2, 3; t = lane % 4, tokens at t/2.
+__device__ __forceinline__ float combine24_lane_factor(int t) { return (t & 1) ? 0.00390625f : 256.0f; }
+
 // Register tables of one (matrix, depth). For depth <= 3, h[0..1] / l[0..1]
 // are the high / low bytes of entries 0..7 (entry v = value of the index whose
 // bit-reversed b-bit form is v). For depth 4, h[0..1] hold entries 0..7 and
@@ -97,9 +132,10 @@ struct RegTab {
 };
 
 // Builds the tables of depth b from the 510-entry codebook; one full warp.
-// big (shared or global, 2^b words) is written for b >= 5 when non-null.
-__device__ __forceinline__ void build_tab(const float *__restrict__ cb, int b, RegTab &tab,
-                                          uint32_t *big)
+// big (shared or global, 2^b entries of 32 or 16 bits: byte 0 = high, byte 1 =
+// low) is written for b >= 5 when non-null.
+template <typename BT = uint32_t>
+__device__ __forceinline__ void build_tab(const float *__restrict__ cb, int b, RegTab &tab, BT *big)
 {
     const int lane = threadIdx.x & 31;
     const int n = 1 << b;
@@ -117,7 +153,7 @@ __device__ __forceinline__ void build_tab(const float *__restrict__ cb, int b, R
         split16(vi, hi, lo);
         const uint32_t e = (uint32_t)(hi & 0xff) | ((uint32_t)(lo & 0xff) << 8);
         if (big != nullptr)
-            big[v] = e;
+            big[v] = (BT)e;
         if (v == lane)
             my = e;
     }
@@ -166,9 +202,9 @@ __device__ __forceinline__ uint32_t tword_hi(const uint32_t (&w)[8][2], int q)
 // A fragments (hi and lo byte planes) of k-step s (0..3) of the lane's tile.
 // ah/al[0]: row g, k 4t..4t+3; [1]: row g+8, same k; [2]: row g, k 16+4t..;
 // [3]: row g+8, k 16+4t.. (PTX m16n8k32 .s8 A layout).
-template <int B>
+template <int B, typename BT = uint32_t>
 __device__ __forceinline__ void decode_kstep(const uint32_t (&w)[8][2], int s, const RegTab &tab,
-                                             const uint32_t *big, uint32_t (&ah)[4],
+                                             const BT *big, uint32_t (&ah)[4],
                                              uint32_t (&al)[4])
 {
 #pragma unroll
@@ -197,10 +233,10 @@ __device__ __forceinline__ void decode_kstep(const uint32_t (&w)[8][2], int s, c
             const uint32_t odd = ((t >> 4) & 0x0f0f0f0fu) | (th & 0xf0f0f0f0u);
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
-                const uint32_t e0 = big[(even >> (16 * hf)) & 0xffu];
-                const uint32_t e1 = big[(odd >> (16 * hf)) & 0xffu];
-                const uint32_t e2 = big[(even >> (16 * hf + 8)) & 0xffu];
-                const uint32_t e3 = big[(odd >> (16 * hf + 8)) & 0xffu];
+                const uint32_t e0 = (uint32_t)big[(even >> (16 * hf)) & 0xffu];
+                const uint32_t e1 = (uint32_t)big[(odd >> (16 * hf)) & 0xffu];
+                const uint32_t e2 = (uint32_t)big[(even >> (16 * hf + 8)) & 0xffu];
+                const uint32_t e3 = (uint32_t)big[(odd >> (16 * hf + 8)) & 0xffu];
                 const uint32_t x01 = prmt(e0, e1, 0x5140u);
                 const uint32_t x23 = prmt(e2, e3, 0x5140u);
                 ah[2 * hf + u] = prmt(x01, x23, 0x5410u);
@@ -256,14 +292,6 @@ __host__ __device__ __forceinline__ void tile_coord(int lane, int q, int j, int 
     const int s = q >> 1, u = q & 1;
     row = g + 8 * u;
     col = 32 * s + 16 * (j >> 2) + 4 * t + (j & 3);
-}
-
-// Combines the four int32 partial sums of one row and one token:
-// dh0 = sum vh*xh, dh1 = sum vh*xl, dl0 = sum vl*xh, dl1 = sum vl*xl.
-__device__ __forceinline__ float combine(int dh0, int dh1, int dl0, int dl1)
-{
-    const int t1 = dh0 * 256 + dh1 + dl0;
-    return __fmaf_rn((float)t1, 256.0f, (float)dl1);
 }
 
 } // namespace dev

@@ -18,8 +18,8 @@ __global__ void __launch_bounds__(128) gemv_kernel(pmoe_matrix m, const void *__
 {
     extern __shared__ __align__(16) unsigned char smem[];
     const int K = m.K, ktiles = K / 128, ng = K / m.G;
-    uint32_t *xf = reinterpret_cast<uint32_t *>(smem);               // [K/32][8][2]
-    int *xe = reinterpret_cast<int *>(xf + (K / 32) * 16);            // [K/128]
+    uint32_t *xf = reinterpret_cast<uint32_t *>(smem);                     // [K/32][24]
+    int *xe = reinterpret_cast<int *>(xf + (K / 32) * dev::kFragWords);     // [K/128]
     uint32_t *big = reinterpret_cast<uint32_t *>(xe + ktiles);        // [256] for B >= 5
     float *red = reinterpret_cast<float *>(big + 256);                // [4][16]
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -31,7 +31,10 @@ __global__ void __launch_bounds__(128) gemv_kernel(pmoe_matrix m, const void *__
     dev::build_tab(m.codebook, B, tab, (B >= 5 && warp == 0) ? big : nullptr);
     __syncthreads();
 
-    const int g = lane >> 2;
+    const int g = lane >> 2, t = lane & 3;
+    // B column g: byte part g of x for g < 3, zero otherwise (xfrag.cuh)
+    const bool fz = g >= 3;
+    const float lf = dev::combine24_lane_factor(t);
     float acc0 = 0.0f, acc1 = 0.0f;
     const float *srow0 = m.scales + (int64_t)(16 * R + g) * ng;
     const float *srow1 = srow0 + 8 * (int64_t)ng;
@@ -48,15 +51,16 @@ __global__ void __launch_bounds__(128) gemv_kernel(pmoe_matrix m, const void *__
                 w[p][1] = v.y;
             }
         }
-        const float fac = ldexpf(1.0f, -(tab.f + xe[Q]));
+        const float fac = lf * ldexpf(1.0f, -(tab.f + xe[Q]));
         int dh[4] = {0, 0, 0, 0}, dl[4] = {0, 0, 0, 0};
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
             uint32_t ah[4], al[4];
             dev::decode_kstep<B>(w, s, tab, big, ah, al);
             uint32_t b0 = 0u, b1 = 0u;
-            if (lane < 8) {
-                const uint2 v = *reinterpret_cast<const uint2 *>(xf + ((Q * 4 + s) * 8 + lane) * 2);
+            if (!fz) {
+                const uint2 v =
+                    *reinterpret_cast<const uint2 *>(xf + (Q * 4 + s) * dev::kFragWords + dev::frag_offset(g, t));
                 b0 = v.x;
                 b1 = v.y;
             }
@@ -64,15 +68,17 @@ __global__ void __launch_bounds__(128) gemv_kernel(pmoe_matrix m, const void *__
             dev::mma_s8(dl, al, b0, b1);
             if ((s + 1) % GS == 0) {
                 const int grp = (128 * Q + 32 * s) / (32 * GS);
-                acc0 = __fmaf_rn(dev::combine(dh[0], dh[1], dl[0], dl[1]), __ldg(srow0 + grp) * fac, acc0);
-                acc1 = __fmaf_rn(dev::combine(dh[2], dh[3], dl[2], dl[3]), __ldg(srow1 + grp) * fac, acc1);
+                acc0 = __fmaf_rn(dev::combine24(dh[0], dh[1], dl[0], dl[1]), __ldg(srow0 + grp) * fac, acc0);
+                acc1 = __fmaf_rn(dev::combine24(dh[2], dh[3], dl[2], dl[3]), __ldg(srow1 + grp) * fac, acc1);
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
                     dh[i] = dl[i] = 0;
             }
         }
     }
-    if ((lane & 3) == 0) {
+    acc0 += __shfl_down_sync(0xffffffffu, acc0, 1);
+    acc1 += __shfl_down_sync(0xffffffffu, acc1, 1);
+    if (t == 0) {
         red[warp * 16 + g] = acc0;
         red[warp * 16 + g + 8] = acc1;
     }
@@ -86,7 +92,7 @@ __global__ void __launch_bounds__(128) gemv_kernel(pmoe_matrix m, const void *__
 template <int B, int GS>
 static pmoe_status launch_gemv_b(const pmoe_matrix &m, const void *x, bool bf, float *y, cudaStream_t st)
 {
-    const size_t smem = (size_t)(m.K / 32) * 64 + (size_t)(m.K / 128) * 4 + 256 * 4 + 64 * 4;
+    const size_t smem = (size_t)(m.K / 32) * dev::kFragWords * 4 + (size_t)(m.K / 128) * 4 + 256 * 4 + 64 * 4;
     if (smem > 200 * 1024)
         return PMOE_ERR_UNSUPPORTED;
     auto kern = bf ? gemv_kernel<B, GS, true> : gemv_kernel<B, GS, false>;

@@ -7,7 +7,7 @@
 //  * xfrag_kernel, only when the batch is too large for the prep kernel to do
 //    it: the activations' MMA fragments.
 //  * layer_prep_kernel (one CTA): routing and selection (decode step), pairs
-//    grouped by expert into column blocks (<= 4 pairs of one depth) and units
+//    grouped by expert into column blocks (<= 2 pairs of one depth) and units
 //    (<= 4 blocks of one expert, deepest units first), one record per unit,
 //    decode tables, activation fragments (small batches) and zeroed counters.
 //  * moe_main_kernel (persistent, one CTA per SM, launched as a programmatic
@@ -55,9 +55,9 @@ LayerWs carve_layer_ws(void *ws, int T, int k, int H, int I, size_t *bytes)
     const size_t o_cb = take(P * (H / 128) * 4), o_yc = take((size_t)T * (H / 128) * 4);
     const size_t o_pa = take(P * (size_t)(I / 16) * 8 * 32 * 4), o_pb = take(P * (size_t)(H / 16) * 2 * 16 * 4);
     const size_t o_tab = take(P * 3 * kTabWords * 4);
-    const size_t o_xf = take((size_t)T * (H / 32) * 16 * 4), o_xe = take((size_t)T * (H / 128) * 4);
+    const size_t o_xf = take((size_t)T * (H / 32) * dev::kFragWords * 4), o_xe = take((size_t)T * (H / 128) * 4);
     const size_t o_h = take(P * I * 4);
-    const size_t o_hf = take(P * (I / 32) * 16 * 4), o_he = take(P * (size_t)hexp_stride(I) * 4);
+    const size_t o_hf = take(P * (I / 32) * dev::kFragWords * 4), o_he = take(P * (size_t)hexp_stride(I) * 4);
     const size_t o_part = take(P * H * 4);
     const size_t o_ids = take(P * 4), o_w = take(P * 4), o_dep = take(P);
     // batch-1 kernel only
@@ -67,6 +67,7 @@ LayerWs carve_layer_ws(void *ws, int T, int k, int H, int I, size_t *bytes)
     const size_t o_pb1 = take(P1 * (H / 16) * nkb * 16 * 4), o_peb = take(P1 * (H / 16) * nkb * 4);
     const size_t o_cb1 = take(P1 * (H / 16) * 4), o_rh = take(P1 * (I / 128) * 4);
     const size_t o_yc1 = take(T == 1 ? (size_t)(H / 16) * 4 : 0);
+    const size_t o_hfl = take(P1 * (I / 16) * 4);
     if (bytes)
         *bytes = off;
     LayerWs L{};
@@ -104,6 +105,7 @@ LayerWs carve_layer_ws(void *ws, int T, int k, int H, int I, size_t *bytes)
     L.cntB1 = reinterpret_cast<int *>(b + o_cb1);
     L.readyH = reinterpret_cast<int *>(b + o_rh);
     L.ycnt1 = reinterpret_cast<int *>(b + o_yc1);
+    L.hflag = reinterpret_cast<int *>(b + o_hfl);
     L.ids = reinterpret_cast<int32_t *>(b + o_ids);
     L.w = reinterpret_cast<float *>(b + o_w);
     L.depth = reinterpret_cast<uint8_t *>(b + o_dep);
@@ -179,7 +181,7 @@ __global__ void __launch_bounds__(kPrepThreads) layer_prep_kernel(PrepArgs a)
         if (a.frags_here) {
             for (int j = wi; j < T * (H / 128); j += nw) {
                 const int t = j / (H / 128), Q = j % (H / 128);
-                dev::make_xfrag_tile<true>(a.x + (int64_t)t * H, Q, W.xfrag + (int64_t)t * (H / 32) * 16,
+                dev::make_xfrag_tile<true>(a.x + (int64_t)t * H, Q, W.xfrag + (int64_t)t * (H / 32) * dev::kFragWords,
                                            W.xexp + (int64_t)t * (H / 128));
             }
         }
@@ -220,7 +222,7 @@ __global__ void __launch_bounds__(kPrepThreads) layer_prep_kernel(PrepArgs a)
             }
             const int e = kk >> 4, d = 15 - (kk & 15);
             const bool new_e = (e != prev_e);
-            if (new_e || d != prev_d || nmem == 4) {
+            if (new_e || d != prev_d || nmem == kMaxMembers) {
                 if (new_e || ublk == kMaxBlocksPerUnit) {
                     u_e[nu] = e;
                     u_b0[nu] = nb;
@@ -299,7 +301,7 @@ __global__ void xfrag_kernel(const uint16_t *__restrict__ x, int T, int H, Layer
     if (gw >= T * (H / 128))
         return;
     const int t = gw / (H / 128), Q = gw % (H / 128);
-    dev::make_xfrag_tile<true>(x + (int64_t)t * H, Q, W.xfrag + (int64_t)t * (H / 32) * 16,
+    dev::make_xfrag_tile<true>(x + (int64_t)t * H, Q, W.xfrag + (int64_t)t * (H / 32) * dev::kFragWords,
                                W.xexp + (int64_t)t * (H / 128));
 }
 
@@ -329,7 +331,7 @@ pmoe_status check_layer(const pmoe_layer *L, int T, int k)
     // an item's scale rows and table heads travel in one ring slot
     if (mk::meta_bytes_gateup(L->H, L->G, kMaxBlocksPerUnit) > mk::CHUNK ||
         mk::meta_bytes_down(L->I, L->G, kMaxBlocksPerUnit) > mk::CHUNK ||
-        mk::meta_bytes_down(L->I, L->G, 1) + mk::meta_bytes_down_frags(L->I, 4) > mk::CHUNK ||
+        mk::meta_bytes_down(L->I, L->G, 1) + mk::meta_bytes_down_frags(L->I, kMaxMembers) > mk::CHUNK ||
         !aligned(L->scales, 16))
         return PMOE_ERR_UNSUPPORTED;
     return PMOE_OK;

@@ -13,6 +13,7 @@ namespace pmoe {
 constexpr int kTabWords = 16 + 256; // h[4], l[4], f, pad | table of 256 entries for depth >= 5
 constexpr int kMaxPairs = 2048;     // T*k per call
 constexpr int kMaxBlocksPerUnit = 4;
+constexpr int kMaxMembers = 2;      // tokens per column block: 3 byte columns each in the 8 of an MMA
 
 // Row stride (ints) of the h-fragment exponents: I/128 rounded up to 16 bytes.
 __host__ __device__ inline int hexp_stride(int I) { return ((I / 128) + 3) & ~3; }
@@ -30,8 +31,8 @@ constexpr int kFlagDone = 7;   // batch-1 kernel: CTAs finished
 // Device pointers into one layer workspace (see carve_layer_ws).
 struct LayerWs {
     int *flags;      // [64]
-    int *blk_depth;  // per column block (<= 4 pairs of one expert and one depth): depth
-    int *blk_nmem;   //   members
+    int *blk_depth;  // per column block (<= 2 pairs of one expert and one depth): depth
+    int *blk_nmem;   //   members (<= kMaxMembers)
     int *blk_pair;   //   [4] pair index t*k + i of each member
     int *blk_expert; //   expert
     int *unit_expert, *unit_blk0, *unit_nblk, *unit_bmax; // per unit (one expert, <= 4 blocks)
@@ -44,10 +45,10 @@ struct LayerWs {
     float *pA;       // [pairs][I/16][8][2][16]: gate/up partial sums per K-part
     float *pB;       // [pairs][H/16][2][16]: down partial sums per K-part
     uint32_t *tabs;  // [pairs][3][kTabWords]: decode tables per block and matrix
-    uint32_t *xfrag; // [T][H/32][8][2]
+    uint32_t *xfrag; // [T][H/32][24]: activation fragments (xfrag.cuh)
     int *xexp;       // [T][H/128]
     float *h;        // [pairs][I]
-    uint32_t *hfrag; // [pairs][I/32][8][2]
+    uint32_t *hfrag; // [pairs][I/32][24]
     int *hexp;       // [pairs][hexp_stride(I)]
     float *part;     // [pairs][H]: down-projection output of each pair
     // batch-1 kernel (T == 1; "pairs" = the k routing slots)
@@ -58,6 +59,7 @@ struct LayerWs {
     int *cntB1;      // [k][H/16]: items of a down row block done
     int *readyH;     // [k][I/128]: 128-row tile of h converted to fragments
     int *ycnt1;      // [H/16]: experts whose rows of this output row block are written
+    int *hflag;      // [k][I/16]: row block of h written in the call whose epoch tag it holds
     int32_t *ids;    // [pairs]: routing results kept by the decode step
     float *w;
     uint8_t *depth;

@@ -42,7 +42,8 @@ constexpr int QDEPTH = 2;                  // item queue (= partial-sum slots): 
 // complete once the current one is claimed, which holds for a two-entry queue.
 static_assert(QDEPTH == 2, "ring slot reuse assumes a two-entry item queue");
 constexpr int RED_WORDS = 16 * 4;          // per warp: [row][member]
-constexpr int XS_WORDS = (4096 / 32) * 16; // shared copy of the x fragments (T == 1, H <= 4096)
+constexpr int KFW = dev::kFragWords;        // words per k-step of a vector's activation fragments
+constexpr int XS_WORDS = (4096 / 32) * dev::kFragWords; // shared copy of the x fragments (T == 1, H <= 4096)
 constexpr int TAB_BYTES = 64;              // decode-table head copied per (block, matrix)
 constexpr uint64_t kDeadlineNs = 200ull * 1000 * 1000;
 
@@ -108,7 +109,7 @@ struct UnitView {
 __host__ __device__ inline int meta_bytes_gateup(int H, int G, int nblk) { return 2 * 16 * (H / G) * 4 + nblk * 2 * TAB_BYTES; }
 __host__ __device__ inline int meta_bytes_down(int I, int G, int nblk) { return 128 * (I / G) * 4 + nblk * TAB_BYTES; }
 // down items with one column block also carry the members' h fragments and exponents
-__host__ __device__ inline int meta_bytes_down_frags(int I, int nmem) { return nmem * (2 * I + hexp_stride(I) * 4); }
+__host__ __device__ inline int meta_bytes_down_frags(int I, int nmem) { return nmem * (3 * I + hexp_stride(I) * 4); }
 
 __device__ __forceinline__ void set_error(const LayerWs &W, int code, int where)
 {
@@ -190,6 +191,7 @@ __device__ __forceinline__ void warp_block(const unsigned char *const (&pp)[8], 
     RegTab tab;
     load_tab_smem(tabs, tab);
     const bool epi = exps != nullptr;
+    const float lf = dev::combine24_lane_factor(threadIdx.x & 3);
     for (int j = 0; j < ntiles; ++j) {
         uint32_t w[8][2];
 #pragma unroll
@@ -201,7 +203,7 @@ __device__ __forceinline__ void warp_block(const unsigned char *const (&pp)[8], 
                 w[p][1] = v.y;
             }
         }
-        const float fac = epi ? 256.0f * pow2neg(tab.f + exp_at<FRAG>(exps + Q0 + j)) : 0.0f;
+        const float fac = epi ? lf * pow2neg(tab.f + exp_at<FRAG>(exps + Q0 + j)) : 0.0f;
         int dh[4] = {0, 0, 0, 0}, dl[4] = {0, 0, 0, 0};
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
@@ -214,8 +216,8 @@ __device__ __forceinline__ void warp_block(const unsigned char *const (&pp)[8], 
             dev::mma_s8(dl, al, bv.x, bv.y);
             if ((s + 1) % GS == 0) {
                 const int gi = j * NG + s / GS;
-                acc0 = __fmaf_rn(combine256(dh[0], dh[1], dl[0], dl[1]), sc0[gi] * fac, acc0);
-                acc1 = __fmaf_rn(combine256(dh[2], dh[3], dl[2], dl[3]), sc1[gi] * fac, acc1);
+                acc0 = __fmaf_rn(dev::combine24(dh[0], dh[1], dl[0], dl[1]), sc0[gi] * fac, acc0);
+                acc1 = __fmaf_rn(dev::combine24(dh[2], dh[3], dl[2], dl[3]), sc1[gi] * fac, acc1);
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
                     dh[i] = dl[i] = 0;
@@ -235,12 +237,13 @@ __device__ __forceinline__ void warp_block_sign(const unsigned char *const (&pp)
     constexpr int NG = 4 / GS;
     const float c1 = __uint_as_float(reinterpret_cast<const uint32_t *>(tabs)[9]);
     const bool epi = exps != nullptr;
+    const float lf = dev::combine24_lane_factor(threadIdx.x & 3);
     for (int j = 0; j < ntiles; ++j) {
         uint32_t w[8][2];
         const uint2 v = *reinterpret_cast<const uint2 *>(pp[0] + j * 256);
         w[0][0] = v.x;
         w[0][1] = v.y;
-        const float fac = epi ? c1 * pow2neg(exp_at<FRAG>(exps + Q0 + j)) : 0.0f;
+        const float fac = epi ? c1 * lf * 0.00390625f * pow2neg(exp_at<FRAG>(exps + Q0 + j)) : 0.0f;
         int dh[4] = {0, 0, 0, 0};
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
@@ -252,8 +255,8 @@ __device__ __forceinline__ void warp_block_sign(const unsigned char *const (&pp)
             dev::mma_s8(dh, a, bv.x, bv.y);
             if ((s + 1) % GS == 0) {
                 const int gi = j * NG + s / GS;
-                acc0 = __fmaf_rn((float)(dh[0] * 256 + dh[1]), sc0[gi] * fac, acc0);
-                acc1 = __fmaf_rn((float)(dh[2] * 256 + dh[3]), sc1[gi] * fac, acc1);
+                acc0 = __fmaf_rn(dev::combine24(dh[0], dh[1], 0, 0), sc0[gi] * fac, acc0);
+                acc1 = __fmaf_rn(dev::combine24(dh[2], dh[3], 0, 0), sc1[gi] * fac, acc1);
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
                     dh[i] = 0;
@@ -283,6 +286,9 @@ __device__ __forceinline__ void warp_block_any(int d, const unsigned char *const
     case 7: warp_block<7, GS, FRAG>(pp, ntiles, Q0, tabs, big, fptr, fstep, exps, sc0, sc1, acc0, acc1); break;
     default: warp_block<8, GS, FRAG>(pp, ntiles, Q0, tabs, big, fptr, fstep, exps, sc0, sc1, acc0, acc1); break;
     }
+    // lanes t = 0, 2 hold tokens 0, 1 of the block once their partners t = 1, 3 are added
+    acc0 += __shfl_down_sync(0xffffffffu, acc0, 1);
+    acc1 += __shfl_down_sync(0xffffffffu, acc1, 1);
 }
 
 // h of one pair, one 128-column tile -> B fragments (one warp); h read through L2.
@@ -293,19 +299,13 @@ __device__ void h_to_frags(const LayerWs &W, int I, int pair, int Q)
     float v[4] = {f.x, f.y, f.z, f.w};
     float m = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
     m = dev::warp_max(m);
-    const int sx = dev::fix_exponent(m);
-    uint32_t ph = 0u, pl = 0u;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        int hi, lo;
-        dev::split16(__float2int_rn(ldexpf(v[i], sx)), hi, lo);
-        ph |= (uint32_t)(hi & 0xff) << (8 * i);
-        pl |= (uint32_t)(lo & 0xff) << (8 * i);
-    }
-    const int s = lane >> 3, o = lane & 7, t = o & 3, reg = o >> 2;
-    uint32_t *xf = W.hfrag + (int64_t)pair * (I / 32) * 16;
-    __stcg(xf + ((Q * 4 + s) * 8 + t) * 2 + reg, ph);
-    __stcg(xf + ((Q * 4 + s) * 8 + 4 + t) * 2 + reg, pl);
+    const int sx = dev::fix_exponent24(m);
+    uint32_t fw[3];
+    dev::frag_words(v, sx, fw);
+    uint32_t *xf = W.hfrag + ((int64_t)pair * (I / 32) + Q * 4) * dev::kFragWords + dev::frag_lane_word(lane);
+    __stcg(xf, fw[0]);
+    __stcg(xf + 8, fw[1]);
+    __stcg(xf + 16, fw[2]);
     if (lane == 0)
         __stcg(W.hexp + (int64_t)pair * hexp_stride(I) + Q, sx);
 }
@@ -529,8 +529,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                 unsigned char *fb = S.ring[s] + sb + nblk * TAB_BYTES;
                 for (int c2 = 0; c2 < nmem; ++c2) {
                     const int pair = UV.bpair(blk0, c2);
-                    pipe::bulk_g2s(fb + c2 * 2 * I, W.hfrag + (int64_t)pair * (I / 32) * 16, 2 * I, bar);
-                    pipe::bulk_g2s(fb + nmem * 2 * I + c2 * hexp_stride(I) * 4,
+                    pipe::bulk_g2s(fb + c2 * 3 * I, W.hfrag + (int64_t)pair * (I / 32) * dev::kFragWords, 3 * I,
+                                   bar);
+                    pipe::bulk_g2s(fb + nmem * 3 * I + c2 * hexp_stride(I) * 4,
                                    W.hexp + (int64_t)pair * hexp_stride(I), hexp_stride(I) * 4, bar);
                 }
             }
@@ -553,7 +554,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
         issue_item(VG, d, 0);
     }
     if (stage_x) {
-        for (int i = tid; i < (H / 32) * 16; i += NTHREADS)
+        for (int i = tid; i < (H / 32) * dev::kFragWords; i += NTHREADS)
             S.xs[i] = W.xfrag[i];
         for (int i = tid; i < H / 128; i += NTHREADS)
             S.xse[i] = W.xexp[i];
@@ -723,34 +724,36 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                 for (int bi = 0; bi < nblk; ++bi) {
                     const int blk = blk0 + bi;
                     const int dd = V.bdepth(blk), nmem = V.bnmem(blk);
-                    const int c = g >> 1;
+                    // B column g = 4*c + part: byte part of token c (part 3 and absent tokens: zero);
+                    // lane t accumulates token t/2 (xfrag.cuh, dev::combine24)
+                    const int c = g >> 2, part = g & 3, me = t >> 1;
+                    const bool has = c < nmem && part < 3;
                     float acc0 = 0.0f, acc1 = 0.0f;
                     const int *exps = nullptr;
-                    if (t < nmem) {
-                        const int tok = V.bpair(blk, t) / k;
+                    if (me < nmem) {
+                        const int tok = V.bpair(blk, me) / k;
                         exps = stage_x ? S.xse : W.xexp + (int64_t)tok * (H / 128);
                     }
                     const unsigned char *tabs = meta + 2 * 16 * ngr * 4 + (bi * 2 + m) * TAB_BYTES;
                     const uint32_t *big = W.tabs + ((int64_t)blk * 3 + m) * kTabWords + 16;
                     if (stage_x) {
-                        const bool has = c < nmem;
-                        const uint32_t *fptr = has ? S.xs + Q0 * 64 + (4 * (g & 1) + t) * 2 : S.zeros;
-                        warp_block_any<GS, 0>(dd, pp, tpw, Q0, tabs, big, fptr, has ? 16 : 0, exps, sc0, sc1, acc0,
+                        const uint32_t *fptr = has ? S.xs + Q0 * 4 * KFW + dev::frag_offset(part, t) : S.zeros;
+                        warp_block_any<GS, 0>(dd, pp, tpw, Q0, tabs, big, fptr, has ? KFW : 0, exps, sc0, sc1, acc0,
                                               acc1);
                     } else {
                         const uint32_t *fptr = nullptr;
-                        if (c < nmem) {
+                        if (has) {
                             const int tok = V.bpair(blk, c) / k;
-                            fptr = W.xfrag + (int64_t)tok * (H / 32) * 16 + Q0 * 64 + (4 * (g & 1) + t) * 2;
+                            fptr = W.xfrag + ((int64_t)tok * (H / 32) + Q0 * 4) * KFW + dev::frag_offset(part, t);
                         }
-                        warp_block_any<GS, 1>(dd, pp, tpw, Q0, tabs, big, fptr, 16, exps, sc0, sc1, acc0, acc1);
+                        warp_block_any<GS, 1>(dd, pp, tpw, Q0, tabs, big, fptr, KFW, exps, sc0, sc1, acc0, acc1);
                     }
-                    if (t < nmem) {
+                    if ((t & 1) == 0 && me < nmem) {
                         if (fast) {
-                            red[g * 4 + t] = acc0;
-                            red[(g + 8) * 4 + t] = acc1;
+                            red[g * 4 + me] = acc0;
+                            red[(g + 8) * 4 + me] = acc1;
                         } else {
-                            const int pair = V.bpair(blk, t);
+                            const int pair = V.bpair(blk, me);
                             float *dst = W.pA + (((int64_t)pair * (I / 16) + d.strip) * 8 + kp) * 32 + m * 16;
                             __stcg(dst + g, acc0);
                             __stcg(dst + g + 8, acc1);
@@ -821,36 +824,37 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
             for (int bi = 0; bi < nblk; ++bi) {
                 const int blk = blk0 + bi;
                 const int dd = V.bdepth(blk), nmem = V.bnmem(blk);
-                const int c = g >> 1;
+                const int c = g >> 2, part = g & 3, me = t >> 1;
+                const bool has = c < nmem && part < 3;
                 float acc0 = 0.0f, acc1 = 0.0f;
                 const unsigned char *tabs = meta + 128 * ngr * 4 + bi * TAB_BYTES;
                 const uint32_t *big = W.tabs + ((int64_t)blk * 3 + 2) * kTabWords + 16;
                 if (fast) {
                     // h fragments and exponents of the members arrived with the meta chunk
                     const uint32_t *hf = reinterpret_cast<const uint32_t *>(meta + 128 * ngr * 4 + TAB_BYTES);
-                    const int *he = reinterpret_cast<const int *>(hf + nmem * (I / 2));
-                    const bool has = c < nmem;
-                    const uint32_t *fptr = has ? hf + c * (I / 2) + Q0 * 64 + (4 * (g & 1) + t) * 2 : S.zeros;
-                    const int *exps = (t < nmem) ? he + t * hexp_stride(I) : nullptr;
-                    warp_block_any<GS, 0>(dd, pp, tpw, Q0, tabs, big, fptr, has ? 16 : 0, exps, sc0, sc1, acc0,
+                    const int *he = reinterpret_cast<const int *>(hf + nmem * (I / 32) * KFW);
+                    const uint32_t *fptr =
+                        has ? hf + ((int64_t)c * (I / 32) + Q0 * 4) * KFW + dev::frag_offset(part, t) : S.zeros;
+                    const int *exps = (me < nmem) ? he + me * hexp_stride(I) : nullptr;
+                    warp_block_any<GS, 0>(dd, pp, tpw, Q0, tabs, big, fptr, has ? KFW : 0, exps, sc0, sc1, acc0,
                                           acc1);
                 } else {
                     const uint32_t *fptr = nullptr;
-                    if (c < nmem) {
+                    if (has) {
                         const int pair = V.bpair(blk, c);
-                        fptr = W.hfrag + (int64_t)pair * (I / 32) * 16 + Q0 * 64 + (4 * (g & 1) + t) * 2;
+                        fptr = W.hfrag + ((int64_t)pair * (I / 32) + Q0 * 4) * KFW + dev::frag_offset(part, t);
                     }
                     const int *exps = nullptr;
-                    if (t < nmem)
-                        exps = W.hexp + (int64_t)V.bpair(blk, t) * hexp_stride(I);
-                    warp_block_any<GS, 2>(dd, pp, tpw, Q0, tabs, big, fptr, 16, exps, sc0, sc1, acc0, acc1);
+                    if (me < nmem)
+                        exps = W.hexp + (int64_t)V.bpair(blk, me) * hexp_stride(I);
+                    warp_block_any<GS, 2>(dd, pp, tpw, Q0, tabs, big, fptr, KFW, exps, sc0, sc1, acc0, acc1);
                 }
-                if (t < nmem) {
+                if ((t & 1) == 0 && me < nmem) {
                     if (fast) {
-                        red[g * 4 + t] = acc0;
-                        red[(g + 8) * 4 + t] = acc1;
+                        red[g * 4 + me] = acc0;
+                        red[(g + 8) * 4 + me] = acc1;
                     } else {
-                        const int pair = V.bpair(blk, t);
+                        const int pair = V.bpair(blk, me);
                         float *dst = W.pB + (((int64_t)pair * (H / 16) + 8 * d.strip + sb) * 2 + kp) * 16;
                         __stcg(dst + g, acc0);
                         __stcg(dst + g + 8, acc1);
