@@ -81,7 +81,7 @@ def peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
 
 
-def traffic_from_profiles(name="decode1_kernel_traffic.txt"):
+def traffic_from_profiles(name="moe_main_kernel_traffic.txt"):
     """Per-launch DRAM bytes of a kernel from its committed ncu summary (None if absent)."""
     p = os.path.join(ROOT, "profiles", name)
     try:
@@ -615,7 +615,7 @@ def main():
         pm.moe_decode_step(R.layer, logits[j], sens, x[j], T, K_TOP, AVG, y[j], ids[j], wts[j], dep[j],
                            ws, ws_bytes, st)
 
-    kernels_per_step = 1  # the batch-1 kernel: route, select, gate/up + SwiGLU, down, combine
+    kernels_per_step = 2  # prep (route, select, group, tables, fragments) + persistent expert kernel
 
     # warm-up (eager)
     for i in range(args.warmup):
@@ -795,7 +795,7 @@ def main():
             "config": layer_config(world),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
-                         "kernel": "decode1_kernel (route, select, gate/up+SwiGLU, down, combine)",
+                         "kernel": "moe_main_kernel (gate/up+SwiGLU, down, combine)",
                          "peak_kind": f"{pk_kind} hbm_gbs"},
             "bitplane_gbs": bitplane_gbs, "bitplane_frac_of_8000": bitplane_gbs / 8000.0,
             "expert_kernels_us": 1e6 * sum(kdur) / len(kdur),

@@ -60,14 +60,6 @@ LayerWs carve_layer_ws(void *ws, int T, int k, int H, int I, size_t *bytes)
     const size_t o_hf = take(P * (I / 32) * dev::kFragWords * 4), o_he = take(P * (size_t)hexp_stride(I) * 4);
     const size_t o_part = take(P * H * 4);
     const size_t o_ids = take(P * 4), o_w = take(P * 4), o_dep = take(P);
-    // batch-1 kernel only
-    const size_t P1 = (T == 1) ? (size_t)k : 0;
-    const size_t nka = (size_t)H / 256, nkb = 8;
-    const size_t o_pa1 = take(P1 * (I / 16) * nka * 32 * 4), o_pea = take(P1 * (I / 16) * nka * 4);
-    const size_t o_pb1 = take(P1 * (H / 16) * nkb * 16 * 4), o_peb = take(P1 * (H / 16) * nkb * 4);
-    const size_t o_cb1 = take(P1 * (H / 16) * 4), o_rh = take(P1 * (I / 128) * 4);
-    const size_t o_yc1 = take(T == 1 ? (size_t)(H / 16) * 4 : 0);
-    const size_t o_hfl = take(P1 * (I / 16) * 4);
     if (bytes)
         *bytes = off;
     LayerWs L{};
@@ -98,14 +90,6 @@ LayerWs carve_layer_ws(void *ws, int T, int k, int H, int I, size_t *bytes)
     L.hfrag = reinterpret_cast<uint32_t *>(b + o_hf);
     L.hexp = reinterpret_cast<int *>(b + o_he);
     L.part = reinterpret_cast<float *>(b + o_part);
-    L.pA1 = reinterpret_cast<float *>(b + o_pa1);
-    L.pendA = reinterpret_cast<int *>(b + o_pea);
-    L.pB1 = reinterpret_cast<float *>(b + o_pb1);
-    L.pendB = reinterpret_cast<int *>(b + o_peb);
-    L.cntB1 = reinterpret_cast<int *>(b + o_cb1);
-    L.readyH = reinterpret_cast<int *>(b + o_rh);
-    L.ycnt1 = reinterpret_cast<int *>(b + o_yc1);
-    L.hflag = reinterpret_cast<int *>(b + o_hfl);
     L.ids = reinterpret_cast<int32_t *>(b + o_ids);
     L.w = reinterpret_cast<float *>(b + o_w);
     L.depth = reinterpret_cast<uint8_t *>(b + o_dep);
@@ -338,6 +322,10 @@ pmoe_status check_layer(const pmoe_layer *L, int T, int k)
 }
 
 static int g_num_sms[128] = {};
+static uint64_t g_wait_limit_ns = 200ull * 1000 * 1000;
+
+void set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns; }
+uint64_t wait_limit_ns() { return g_wait_limit_ns; }
 
 pmoe_status launch_layer(const pmoe_layer *L, const float *logits, const float *sens, const uint16_t *x,
                          int32_t *ids, float *w, uint8_t *depth, int T, int k, int B, float *y, void *ws,
@@ -348,8 +336,6 @@ pmoe_status launch_layer(const pmoe_layer *L, const float *logits, const float *
     if (ws_bytes < need)
         return PMOE_ERR_WORKSPACE;
     LayerWs W = carve_layer_ws(ws, T, k, L->H, L->I, nullptr);
-    if (T == 1)
-        return launch_decode1(L, logits, sens, x, ids, w, depth, k, B, y, W, st, g_prof_start, g_prof_stop);
     const int P = T * k;
     const bool frags_here = (int64_t)T * (L->H / 128) <= 128;
     if (!frags_here) {

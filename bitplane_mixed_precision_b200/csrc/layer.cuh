@@ -24,9 +24,6 @@ constexpr int kFlagBlocks = 1; // column blocks
 constexpr int kFlagUnits = 2;  // expert units
 constexpr int kFlagSched = 3;  // work counter of the persistent kernel
 constexpr int kFlagWhere = 4;  // detail of the first error
-constexpr int kFlagSeq = 5;    // batch-1 kernel: call epoch of this workspace (advanced by the last CTA)
-constexpr int kFlagGo = 6;     // batch-1 kernel: epoch tag published once the call's counters are reset
-constexpr int kFlagDone = 7;   // batch-1 kernel: CTAs finished
 
 // Device pointers into one layer workspace (see carve_layer_ws).
 struct LayerWs {
@@ -51,15 +48,6 @@ struct LayerWs {
     uint32_t *hfrag; // [pairs][I/32][24]
     int *hexp;       // [pairs][hexp_stride(I)]
     float *part;     // [pairs][H]: down-projection output of each pair
-    // batch-1 kernel (T == 1; "pairs" = the k routing slots)
-    float *pA1;      // [k][I/16][H/256][32]: gate/up row sums of row-block pieces split between CTAs
-    int *pendA;      // [k][I/16][H/256]: end (item) of the piece starting there
-    float *pB1;      // [k][H/16][<=8][16]: down row sums of split row-block pieces
-    int *pendB;      // [k][H/16][<=8]
-    int *cntB1;      // [k][H/16]: items of a down row block done
-    int *readyH;     // [k][I/128]: 128-row tile of h converted to fragments
-    int *ycnt1;      // [H/16]: experts whose rows of this output row block are written
-    int *hflag;      // [k][I/16]: row block of h written in the call whose epoch tag it holds
     int32_t *ids;    // [pairs]: routing results kept by the decode step
     float *w;
     uint8_t *depth;
@@ -73,10 +61,6 @@ pmoe_status launch_layer(const pmoe_layer *L, const float *logits, const float *
                          int32_t *ids, float *w, uint8_t *depth, int T, int k, int B, float *y, void *ws,
                          size_t ws_bytes, cudaStream_t st);
 
-// The batch-1 kernel (one launch: routing, selection, gate/up + SwiGLU, down, combine).
-pmoe_status launch_decode1(const pmoe_layer *L, const float *logits, const float *sens, const uint16_t *x,
-                           int32_t *ids, float *w, uint8_t *depth, int k, int B, float *y, const LayerWs &W,
-                           cudaStream_t st, cudaEvent_t ev0, cudaEvent_t ev1);
 // Limit of every bounded wait inside the layer kernels (one deadline per launch).
 void set_wait_limit_ns(uint64_t ns);
 uint64_t wait_limit_ns();

@@ -62,14 +62,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 }
 
 // Waits for the phase with the given parity to complete; false if the
-// deadline (global timer, ns) passed first.
+// deadline (global timer, ns) passed first. After a few quick tests the thread
+// sleeps between tests (up to 256 ns), so that waiting warps leave the issue
+// slots to the warps that compute.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t deadline)
 {
-    for (;;) {
+    uint32_t ns = 16;
+    for (int it = 0;; ++it) {
         if (mbar_try_wait(bar, parity))
             return true;
-        if (globaltimer() > deadline)
+        if ((it & 7) == 0 && globaltimer() > deadline)
             return false;
+        if (it >= 2) {
+            __nanosleep(ns);
+            ns = ns < 256 ? 2 * ns : 256;
+        }
     }
 }
 

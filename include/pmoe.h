@@ -315,9 +315,7 @@ PMOE_API pmoe_status pmoe_moe_layer_fwd_noalloc(const pmoe_layer *L, const uint1
  * pmoe_layer_error: reads the device-side error record of the last layer call
  * that used workspace ws (synchronises the stream). code: 0 none, 1 expert id
  * or depth out of range, 2 a needed plane has no slot (detail = e*8 + plane),
- * 3 a bounded wait inside the kernel ran out (detail = where), 4 a batch-1
- * call whose routing leaves one SM more than four experts' down rows (the
- * kernel's h staging; not reachable with k <= 32 on 148 SMs).
+ * 3 a bounded wait inside the kernel ran out (detail = where).
  */
 PMOE_API pmoe_status pmoe_layer_error(const void *ws, int *code, int *detail, pmoe_stream stream);
 
@@ -326,7 +324,8 @@ PMOE_API pmoe_status pmoe_layer_error(const void *ws, int *code, int *detail, pm
  * later pmoe_moe_layer_fwd / pmoe_moe_decode_step calls (process-wide): each
  * launch gives up on any wait once this many nanoseconds have passed since it
  * started, records error 3 (see pmoe_layer_error) and finishes. Waits for the
- * kernel's own copies to land before it exits use a separate 1 s bound.
+ * kernel's own copies to land before it exits have a separate bound, 200 ms
+ * past that one.
  * 0 restores the default of 200 ms. Host only; the kernels stay correct with
  * any limit that is not reached.
  */
