@@ -71,6 +71,8 @@ _SIGS = {
     "pmoe_noalloc_layer_error": ([ctypes.POINTER(i32), ctypes.POINTER(i32), P], i32),
     "pmoe_moe_layer_fwd_noalloc": ([ctypes.POINTER(Layer), P, P, P, P, i32, i32, P, P], i32),
     "pmoe_layer_error": ([P, ctypes.POINTER(i32), ctypes.POINTER(i32), P], i32),
+    "pmoe_layer_counts": ([P, P, P], i32),
+    "pmoe_tc_selfcheck": ([P, P, P, i32, i32, P], i32),
     "pmoe_set_wait_limit_ns": ([ctypes.c_uint64], i32),
     "pmoe_materialise_workspace_bytes": ([i32, i32, i32, i32, i32], sz),
     "pmoe_materialise_layer_fwd": ([ctypes.POINTER(Layer), P, P, P, P, i32, i32, P, P, sz, P], i32),
@@ -264,6 +266,20 @@ def layer_error(ws, stream=None):
     _check("pmoe_layer_error", _lib.pmoe_layer_error(_ptr(ws), ctypes.byref(code), ctypes.byref(detail),
                                                      _stream(stream)))
     return code.value, detail.value
+
+
+def layer_counts(ws, stream=None):
+    """(column blocks, expert units, tensor-core units, tensor-core operand rows) of the last layer
+    call on workspace ws (synchronises)."""
+    out = (i32 * 4)()
+    _check("pmoe_layer_counts", _lib.pmoe_layer_counts(_ptr(ws), out, _stream(stream)))
+    return tuple(out)
+
+
+def tc_selfcheck(A, B, D, N, K, stream=None) -> None:
+    """D[128 x N] = A[128 x K] * B[N x K]^T through the tensor-core operand path (f16 bit patterns as
+    int16 tensors, D fp32)."""
+    _check("pmoe_tc_selfcheck", _lib.pmoe_tc_selfcheck(_ptr(A), _ptr(B), _ptr(D), N, K, _stream(stream)))
 
 
 def materialise_workspace_bytes(T, k, E, H, I) -> int:

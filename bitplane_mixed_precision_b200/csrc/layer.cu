@@ -60,6 +60,12 @@ LayerWs carve_layer_ws(void *ws, int T, int k, int H, int I, size_t *bytes)
     const size_t o_hf = take(P * (I / 32) * dev::kFragWords * 4), o_he = take(P * (size_t)hexp_stride(I) * 4);
     const size_t o_part = take(P * H * 4);
     const size_t o_ids = take(P * 4), o_w = take(P * 4), o_dep = take(P);
+    // tensor-core path
+    const bool tc = T >= kTcMinTokens;
+    const size_t R = tc ? (size_t)tc_max_rows((int)P) : 0, U = tc ? P / kTcMinTokens + 1 : 0;
+    const size_t o_tu = take(U * 16), o_trp = take(R * 4), o_trd = take(R * 4), o_tru = take(R * 4);
+    const size_t o_trx = take(R * 4), o_trh = take(R * 4);
+    const size_t o_txb = take(R * H * 2), o_thb = take(R * I * 2), o_tgu = take(tc ? P * 2 * I * 4 : 0);
     if (bytes)
         *bytes = off;
     LayerWs L{};
@@ -90,6 +96,17 @@ LayerWs carve_layer_ws(void *ws, int T, int k, int H, int I, size_t *bytes)
     L.hfrag = reinterpret_cast<uint32_t *>(b + o_hf);
     L.hexp = reinterpret_cast<int *>(b + o_he);
     L.part = reinterpret_cast<float *>(b + o_part);
+    if (tc) {
+        L.tc_unit = reinterpret_cast<int4 *>(b + o_tu);
+        L.tc_rpair = reinterpret_cast<int *>(b + o_trp);
+        L.tc_rdep = reinterpret_cast<int *>(b + o_trd);
+        L.tc_runit = reinterpret_cast<int *>(b + o_tru);
+        L.tc_rxe = reinterpret_cast<int *>(b + o_trx);
+        L.tc_rhe = reinterpret_cast<int *>(b + o_trh);
+        L.tc_xb = reinterpret_cast<uint16_t *>(b + o_txb);
+        L.tc_hb = reinterpret_cast<uint16_t *>(b + o_thb);
+        L.tc_gu = reinterpret_cast<float *>(b + o_tgu);
+    }
     L.ids = reinterpret_cast<int32_t *>(b + o_ids);
     L.w = reinterpret_cast<float *>(b + o_w);
     L.depth = reinterpret_cast<uint8_t *>(b + o_dep);
@@ -113,6 +130,7 @@ struct PrepArgs {
     float *w;
     uint8_t *depth;
     int frags_here; // 1: this kernel converts x; 0: a separate grid kernel did
+    int tc;         // 1: experts hit by enough pairs go to the tensor-core units
     int n_rw;       // routing warps (decode step), each with E floats of staging
     LayerWs W;
 };
@@ -196,9 +214,52 @@ __global__ void __launch_bounds__(kPrepThreads) layer_prep_kernel(PrepArgs a)
     int *u_e = sm + 2 * P, *u_b0 = sm + 3 * P, *u_nb = sm + 4 * P, *u_bm = sm + 5 * P;
     __shared__ int s_nb, s_nu;
     if (tid == 0) {
+        // 2a. tensor-core units: an expert whose pairs at depth <= kTcMaxLevels number at least
+        //     kTcMinTokens gives them to units of at most kTcMaxCols pairs (the pairs of a run of one
+        //     expert are ordered by depth, deepest first, so they are the run's tail); its deeper pairs
+        //     stay with the persistent kernel. Operand rows: a unit's pairs, then zero rows up to a
+        //     multiple of 16.
+        int ntc = 0, nrow = 0;
+        if (a.tc) {
+            for (int r0 = 0; r0 < P;) {
+                const int k0 = key[sorted[r0]];
+                int r1 = r0 + 1;
+                while (r1 < P && k0 >= 0 && (key[sorted[r1]] >> 4) == (k0 >> 4))
+                    ++r1;
+                if (k0 >= 0) {
+                    int rs = r0;
+                    while (rs < r1 && 15 - (key[sorted[rs]] & 15) > kTcMaxLevels)
+                        ++rs;
+                    const int cnt = r1 - rs;
+                    if (cnt >= kTcMinTokens) {
+                        const int nun = (cnt + kTcMaxCols - 1) / kTcMaxCols;
+                        for (int j = 0, r = rs; j < nun; ++j) {
+                            const int n = cnt / nun + (j < cnt % nun ? 1 : 0), npad = (n + 15) & ~15;
+                            const int bmax = 15 - (key[sorted[r]] & 15);
+                            W.tc_unit[ntc] = make_int4(k0 >> 4, n, npad | (bmax << 16), nrow);
+                            for (int c = 0; c < npad; ++c, ++nrow) {
+                                const int pr = c < n ? sorted[r + c] : -1;
+                                W.tc_rpair[nrow] = pr;
+                                W.tc_rdep[nrow] = pr >= 0 ? 15 - (key[pr] & 15) : 0;
+                                W.tc_runit[nrow] = ntc;
+                            }
+                            for (int c = 0; c < n; ++c)
+                                sorted[r + c] = -1; // leaves the persistent kernel's blocks
+                            r += n;
+                            ++ntc;
+                        }
+                    }
+                }
+                r0 = r1;
+            }
+        }
+        W.flags[kFlagTcUnits] = ntc;
+        W.flags[kFlagTcRows] = nrow;
         int nb = 0, nu = 0, prev_e = -1, prev_d = -1, nmem = 0, ublk = 0, bad = 0;
         for (int r = 0; r < P; ++r) {
             const int p = sorted[r];
+            if (p < 0)
+                continue;
             const int kk = key[p];
             if (kk < 0) {
                 bad = 1;
@@ -352,13 +413,17 @@ pmoe_status launch_layer(const pmoe_layer *L, const float *logits, const float *
         n_rw = n_rw < cap ? n_rw : cap;
         n_rw = n_rw > 1 ? n_rw : 1;
     }
-    PrepArgs pa{*L, logits, sens, x, T, k, B, ids, w, depth, frags_here ? 1 : 0, n_rw, W};
+    // (the tensor-core kernels stage 128 rows x K/G scales of at most 32 groups)
+    const bool tc = W.tc_unit != nullptr && L->H / L->G <= 32 && L->I / L->G <= 32;
+    PrepArgs pa{*L, logits, sens, x, T, k, B, ids, w, depth, frags_here ? 1 : 0, tc ? 1 : 0, n_rw, W};
     const size_t prep_smem = 6 * (size_t)P * sizeof(int) + (size_t)n_rw * L->E * sizeof(float);
     if (prep_smem > 40 * 1024)
         PMOE_CUDA(cudaFuncSetAttribute(layer_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_smem));
     layer_prep_kernel<<<1, kPrepThreads, prep_smem, st>>>(pa);
     PMOE_TRY(launch_status());
 
+    if (tc)
+        PMOE_TRY(launch_tc(L, x, w, T, k, y, W, st));
     int dev = 0;
     PMOE_CUDA(cudaGetDevice(&dev));
     if (dev < 0 || dev >= 128)
@@ -433,6 +498,20 @@ pmoe_status pmoe_layer_error(const void *ws, int *code, int *detail, pmoe_stream
     *code = f[kFlagError];
     if (detail)
         *detail = f[kFlagWhere];
+    return PMOE_OK;
+}
+
+pmoe_status pmoe_layer_counts(const void *ws, int *counts, pmoe_stream stream)
+{
+    if (!ws || !counts)
+        return PMOE_ERR_INVALID_ARG;
+    int f[16];
+    PMOE_CUDA(cudaMemcpyAsync(f, ws, sizeof(f), cudaMemcpyDeviceToHost, (cudaStream_t)stream));
+    PMOE_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
+    counts[0] = f[kFlagBlocks];
+    counts[1] = f[kFlagUnits];
+    counts[2] = f[kFlagTcUnits];
+    counts[3] = f[kFlagTcRows];
     return PMOE_OK;
 }
 

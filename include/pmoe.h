@@ -312,6 +312,29 @@ PMOE_API pmoe_status pmoe_moe_layer_fwd_noalloc(const pmoe_layer *L, const uint1
                                                 pmoe_stream stream);
 
 /*
+ * pmoe_layer_counts: how the last layer call that used workspace ws grouped
+ * its pairs (synchronises the stream): counts[0] column blocks and counts[1]
+ * expert units of the persistent kernel, counts[2] tensor-core units (experts
+ * hit by at least 8 pairs at depth <= 4, batches of T >= 8 tokens), counts[3]
+ * their operand rows (pairs padded to multiples of 16 per unit).
+ */
+PMOE_API pmoe_status pmoe_layer_counts(const void *ws, int *counts, pmoe_stream stream);
+
+/*
+ * pmoe_tc_selfcheck: checks the tensor-core operand path that the batched
+ * layer uses for experts hit by many tokens (tcgen05 MMA, f16 operands in
+ * shared memory, fp32 accumulator in tensor memory). Computes
+ * D[128 x N] = A[128 x K] * B[N x K]^T on the device with the same operand
+ * layout, descriptors, MMA, completion and tensor-memory loads as the layer's
+ * kernel. A, B: device, row-major f16 (bit patterns as uint16), 16-byte
+ * aligned; D: device fp32, row-major. 16 <= N <= 64, N % 16 == 0;
+ * 32 <= K <= 128, K % 32 == 0. Asynchronous on stream; INVALID_ARG for other
+ * shapes or null pointers.
+ */
+PMOE_API pmoe_status pmoe_tc_selfcheck(const uint16_t *A, const uint16_t *B, float *D, int N, int K,
+                                       pmoe_stream stream);
+
+/*
  * pmoe_layer_error: reads the device-side error record of the last layer call
  * that used workspace ws (synchronises the stream). code: 0 none, 1 expert id
  * or depth out of range, 2 a needed plane has no slot (detail = e*8 + plane),

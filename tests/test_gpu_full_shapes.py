@@ -109,6 +109,27 @@ def test_large_layer_zipf_batch_of_32(pm, big):
         assert_close(y[t], ref[t], msg=f"token {t}")
 
 
+@pytest.mark.parametrize("T", [64, 128])
+def test_large_layer_zipf_batches_of_64_and_128(pm, big, T):
+    """Larger Zipf(1.1)-biased batches: the popular experts go to the tensor-core units (one
+    accumulator per tree level, up to 64 pairs each); routing and selection bit-exact, a sample of
+    tokens (those with the most tensor-core pairs and a few others) element-wise against the oracle."""
+    R, O = big
+    sens = synth.sensitivities(SEED, 0, E)
+    bias = synth.zipf_bias(SEED, E)
+    logits, xb = tokens(SEED, T, E, H, token0=1000 + T, bias=bias)
+    y, ids, w, dep = _decode(pm, R, logits, xb, sens, T)
+    _check_routing(logits, sens, ids, w, dep)
+    shallow = np.bincount(ids[dep <= 4], minlength=E)
+    hot = shallow >= 8
+    assert hot.sum() >= 4
+    n_tc = (hot[ids] & (dep <= 4)).sum(axis=1)
+    sample = sorted(set(np.argsort(-n_tc, kind="stable")[:6].tolist()) | {0, T // 2, T - 1})
+    ref = O.run(E, ids[sample], w[sample], dep[sample], synth.bf16_to_f32(xb[sample]).astype(np.float64))
+    for j, t in enumerate(sample):
+        assert_close(y[t], ref[j], msg=f"token {t}")
+
+
 L_STACK = 16
 
 
