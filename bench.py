@@ -504,53 +504,92 @@ def batch_bench(args):
         per_exp.append(Tb * K_TOP / len(bmax))
     achieved = float(sum(alg) / sum(kdur)) / 1e9
     pk, pk_kind = peaks()
-    # graph-captured timed steps
+    # tensor-core units of each batch (experts with >= 8 pairs at depth <= 4, units of <= 32 pairs):
+    # counted by the library, and their MMA work (2 parts x levels x 2 flop per weight and token)
+    tc_units, tc_rows, tc_pairs, tc_flop = [], [], [], []
+    for b in range(nb):
+        step(b, st)
+        cnt = pm.layer_counts(ws)
+        tc_units.append(cnt[2])
+        tc_rows.append(cnt[3])
+        pairs, flop = 0, 0.0
+        for e in np.unique(ids_h[b]):
+            sel = (ids_h[b] == e) & (dep_h[b] <= 4)
+            n = int(sel.sum())
+            if n < 8:
+                continue
+            pairs += n
+            d = np.sort(dep_h[b][sel])[::-1]
+            nun = (n + 31) // 32
+            for j, start in enumerate(np.cumsum([0] + [n // nun + (1 if i < n % nun else 0) for i in range(nun)])[:-1]):
+                m = n // nun + (1 if j < n % nun else 0)
+                npad = (m + 15) // 16 * 16
+                nlev = int(d[start])
+                flop += 2.0 * 2 * nlev * npad * 3 * H * I
+        tc_pairs.append(pairs)
+        tc_flop.append(flop)
+
+    def timed_steps():
+        steps = args.steps
+        cap = torch.cuda.Stream(dev)
+        gsize = min(steps, 1024)
+        graphs = []
+        for g0 in range(0, steps, gsize):
+            n = min(gsize, steps - g0)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                for i in range(n):
+                    step(g0 + i, cap)
+            graphs.append((g, n))
+        for g, _ in graphs[:1]:
+            g.replay()
+        torch.cuda.synchronize()
+        clk = ClockSampler(gpu_bus_id(dev))
+        clk.start()
+        a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for g, _ in graphs:
+            g.replay()
+        b2.record()
+        torch.cuda.synchronize()
+        clocks = clk.stop()
+        t = a.elapsed_time(b2) * 1e-3
+        for g, _ in graphs:
+            del g
+        graphs.clear()
+        return t, clocks
+
     steps = args.steps
-    cap = torch.cuda.Stream(dev)
-    gsize = min(steps, 1024)
-    graphs = []
-    for g0 in range(0, steps, gsize):
-        n = min(gsize, steps - g0)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=cap):
-            for i in range(n):
-                step(g0 + i, cap)
-        graphs.append((g, n))
-    for g, _ in graphs[:1]:
-        g.replay()
-    torch.cuda.synchronize()
-    clk = ClockSampler(gpu_bus_id(dev))
-    clk.start()
-    a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for g, _ in graphs:
-        g.replay()
-    b2.record()
-    torch.cuda.synchronize()
-    clocks = clk.stop()
-    t = a.elapsed_time(b2) * 1e-3
-    for g, _ in graphs:
-        del g
-    graphs.clear()
+    t, clocks = timed_steps()
+    # the same batches with every pair on the persistent kernel (no tensor-core units), for comparison
+    pm.set_tc_min_tokens(0)
+    try:
+        t_nt, _ = timed_steps()
+    finally:
+        pm.set_tc_min_tokens(8)
     line = {
         "metric": f"batched MoE-layer decode tokens/s ({Tb} tokens per step)", "value": steps * Tb / t,
         "unit": "tokens/s", "n_gpus": 1, "steps": steps, "warmup": max(args.warmup, nb),
         "ms_per_step": t * 1e3 / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "s8 mma / s32 acc / f32", "data": "synthetic",
+        "dtype": "s8 mma.sync + f16 tcgen05 / f32 acc", "data": "synthetic",
         "config": {"workload": f"moe_layer_e{E}_top10_h4096_i1024_g128_avg2.5_batch{Tb}_zipf1.1",
                    "experts": E, "top_k": K_TOP, "batch": Tb, "batches_distinct": nb,
                    "l2": "inputs larger than L2 (6.4 GB of resident planes), fresh batch per step; "
                          "kernel timing with L2 flushed before each batch"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / pk["hbm_gbs"], "traffic": None,
-                     "kernel": "moe_main_kernel (gate/up+SwiGLU, down, combine)",
+                     "kernel": "tensor-core kernels + moe_main_kernel (gate/up+SwiGLU, down, combine)",
                      "peak_kind": f"{pk_kind} hbm_gbs"},
         "expert_kernels_us": 1e6 * sum(kdur) / nb,
+        "tensor_core": {"units": float(np.mean(tc_units)), "operand_rows": float(np.mean(tc_rows)),
+                        "pairs": float(np.mean(tc_pairs)), "pairs_frac": float(np.mean(tc_pairs)) / (Tb * K_TOP),
+                        "mma_gflop_per_batch": float(np.mean(tc_flop)) / 1e9},
+        "persistent_only": {"tokens_per_s": steps * Tb / t_nt, "ms_per_step": t_nt * 1e3 / steps},
         "per_batch": {"distinct_experts": float(np.mean(n_exp)), "pairs_per_expert": float(np.mean(per_exp)),
                       "plane_bytes": float(np.mean(plane_b)), "algorithmic_bytes": float(np.mean(alg)),
                       "mean_bits": float(dep_h.mean())},
         "layer_error": list(err),
-        "gpu_launches": steps * 3,  # x fragments, prep, expert kernel
+        "gpu_launches": steps * 7,  # x fragments, prep, 4 tensor-core kernels, persistent expert kernel
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

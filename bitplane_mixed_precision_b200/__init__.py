@@ -72,6 +72,7 @@ _SIGS = {
     "pmoe_moe_layer_fwd_noalloc": ([ctypes.POINTER(Layer), P, P, P, P, i32, i32, P, P], i32),
     "pmoe_layer_error": ([P, ctypes.POINTER(i32), ctypes.POINTER(i32), P], i32),
     "pmoe_layer_counts": ([P, P, P], i32),
+    "pmoe_set_tc_min_tokens": ([i32], i32),
     "pmoe_tc_selfcheck": ([P, P, P, i32, i32, P], i32),
     "pmoe_set_wait_limit_ns": ([ctypes.c_uint64], i32),
     "pmoe_materialise_workspace_bytes": ([i32, i32, i32, i32, i32], sz),
@@ -274,6 +275,11 @@ def layer_counts(ws, stream=None):
     out = (i32 * 4)()
     _check("pmoe_layer_counts", _lib.pmoe_layer_counts(_ptr(ws), out, _stream(stream)))
     return tuple(out)
+
+
+def set_tc_min_tokens(n) -> None:
+    """Pairs at depth <= 4 an expert needs in one call before the tensor cores take them (>= 8; 0: never)."""
+    _check("pmoe_set_tc_min_tokens", _lib.pmoe_set_tc_min_tokens(int(n)))
 
 
 def tc_selfcheck(A, B, D, N, K, stream=None) -> None:

@@ -130,7 +130,8 @@ struct PrepArgs {
     float *w;
     uint8_t *depth;
     int frags_here; // 1: this kernel converts x; 0: a separate grid kernel did
-    int tc;         // 1: experts hit by enough pairs go to the tensor-core units
+    int tc;         // > 0: experts with at least this many pairs at depth <= kTcMaxLevels go to the
+                    // tensor-core units (0: none)
     int n_rw;       // routing warps (decode step), each with E floats of staging
     LayerWs W;
 };
@@ -231,7 +232,7 @@ __global__ void __launch_bounds__(kPrepThreads) layer_prep_kernel(PrepArgs a)
                     while (rs < r1 && 15 - (key[sorted[rs]] & 15) > kTcMaxLevels)
                         ++rs;
                     const int cnt = r1 - rs;
-                    if (cnt >= kTcMinTokens) {
+                    if (cnt >= a.tc) {
                         const int nun = (cnt + kTcMaxCols - 1) / kTcMaxCols;
                         for (int j = 0, r = rs; j < nun; ++j) {
                             const int n = cnt / nun + (j < cnt % nun ? 1 : 0), npad = (n + 15) & ~15;
@@ -384,6 +385,7 @@ pmoe_status check_layer(const pmoe_layer *L, int T, int k)
 
 static int g_num_sms[128] = {};
 static uint64_t g_wait_limit_ns = 200ull * 1000 * 1000;
+static int g_tc_min = kTcMinTokens;
 
 void set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns; }
 uint64_t wait_limit_ns() { return g_wait_limit_ns; }
@@ -413,15 +415,18 @@ pmoe_status launch_layer(const pmoe_layer *L, const float *logits, const float *
         n_rw = n_rw < cap ? n_rw : cap;
         n_rw = n_rw > 1 ? n_rw : 1;
     }
-    // (the tensor-core kernels stage 128 rows x K/G scales of at most 32 groups)
-    const bool tc = W.tc_unit != nullptr && L->H / L->G <= 32 && L->I / L->G <= 32;
-    PrepArgs pa{*L, logits, sens, x, T, k, B, ids, w, depth, frags_here ? 1 : 0, tc ? 1 : 0, n_rw, W};
+    // (the tensor-core epilogue reads one scale per group: at most 32 groups along K keep the
+    // group accumulators' turnover below the decode rate)
+    const bool tc = W.tc_unit != nullptr && g_tc_min > 0 && L->H / L->G <= 32 && L->I / L->G <= 32;
+    PrepArgs pa{*L, logits, sens, x, T, k, B, ids, w, depth, frags_here ? 1 : 0, tc ? g_tc_min : 0, n_rw, W};
     const size_t prep_smem = 6 * (size_t)P * sizeof(int) + (size_t)n_rw * L->E * sizeof(float);
     if (prep_smem > 40 * 1024)
         PMOE_CUDA(cudaFuncSetAttribute(layer_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_smem));
     layer_prep_kernel<<<1, kPrepThreads, prep_smem, st>>>(pa);
     PMOE_TRY(launch_status());
 
+    if (g_prof_start)
+        PMOE_CUDA(cudaEventRecord(g_prof_start, st));
     if (tc)
         PMOE_TRY(launch_tc(L, x, w, T, k, y, W, st));
     int dev = 0;
@@ -449,8 +454,6 @@ pmoe_status launch_layer(const pmoe_layer *L, const float *logits, const float *
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (g_prof_start)
-        PMOE_CUDA(cudaEventRecord(g_prof_start, st));
     PMOE_CUDA(cudaLaunchKernelEx(&cfg, kern, ma));
     if (g_prof_stop)
         PMOE_CUDA(cudaEventRecord(g_prof_stop, st));
@@ -498,6 +501,14 @@ pmoe_status pmoe_layer_error(const void *ws, int *code, int *detail, pmoe_stream
     *code = f[kFlagError];
     if (detail)
         *detail = f[kFlagWhere];
+    return PMOE_OK;
+}
+
+pmoe_status pmoe_set_tc_min_tokens(int n)
+{
+    if (n != 0 && n < kTcMinTokens)
+        return PMOE_ERR_INVALID_ARG;
+    g_tc_min = n;
     return PMOE_OK;
 }
 

@@ -3,17 +3,18 @@
 // multiplied on the fifth-generation tensor cores (tcgen05) instead of being
 // decoded again for every pair of tokens.
 //
-// For such an expert ("TC unit": one expert, up to 64 of its (token, slot)
+// For such an expert ("TC unit": one expert, up to 32 of its (token, slot)
 // pairs, all at depth <= 4) the tree value at depth b is written as a sum of
 // level deltas (children = parent + delta):
 //     C_b[i] = sum_{d=1..b} Delta_d[i >> (b-d)],  Delta_1 = C_1,
 //     Delta_d[j] = C_d[j] - C_{d-1}[j >> 1],
 // and every level d has its own accumulator. A 128-row tile of a matrix is
-// decoded once per level into f16 operands in shared memory (each table entry
-// Delta_d * 2^fa split into a high and a low f16 part, two MMAs, so that the
-// entries are exact to about 2^-22 and no rounding error repeats across the
-// many weights that share an entry), and one MMA per level and part multiplies
-// it with all the unit's tokens at once. Accumulators hold one scale group
+// decoded once per level into f16 operands in shared memory, and one MMA per
+// level multiplies it with all the unit's tokens at once. The entries of level
+// 1, the largest deltas, are split into a high and a low f16 part (two MMAs):
+// one f16 per entry repeats the entry's rounding error on every weight that
+// uses it, and those errors add up coherently in a dot product; for levels
+// 2..4 (smaller deltas) the single f16 stays inside the layer's tolerance. Accumulators hold one scale group
 // (G columns of K) at a time; the epilogue applies the rows' group scales in
 // fp32 and sums, per token, the first b level accumulators of its depth b.
 // Tokens at different depths of one expert thus share the planes they have in
@@ -58,7 +59,7 @@ constexpr int KCH = 128;                                     // k per ring chunk
 constexpr int KS_CH = KCH / 32;                              // k-steps per chunk
 constexpr int NSLOT = 2, NST = 2;                            // ring slots, decoded stages
 constexpr int PLANES_CH = NDEC * kTcMaxLevels * 256;         // plane tiles of a chunk (8 KB)
-constexpr int BOPS_CH = KS_CH * kTcMaxCols * 64;             // B operand of a chunk (16 KB)
+constexpr int BOPS_CH = KS_CH * kTcMaxCols * 64;             // B operand of a chunk (8 KB)
 constexpr int SLOT_BYTES = PLANES_CH + BOPS_CH;
 constexpr int LEV_BYTES = 128 * 32 * 2;                      // one level part of a decoded k-step
 constexpr int STAGE_BYTES = kTcMaxLevels * 2 * LEV_BYTES;    // levels x (high, low parts)
@@ -251,17 +252,18 @@ __device__ __forceinline__ void decode_kstep(const uint32_t (&w)[kTcMaxLevels][2
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 const uint32_t sel = hf ? (tw >> 16) : tw;
-                uint32_t h01, h23, l01, l23;
-                if (d >= 3) {
+                uint32_t h01, h23;
+                if (d >= 3)
                     lookup4<true>(tb[d], sel, h01, h23);
-                    lookup4<true>(tb[d] + 8, sel, l01, l23);
-                } else {
+                else
                     lookup4<false>(tb[d], sel, h01, h23);
-                    lookup4<false>(tb[d] + 8, sel, l01, l23);
-                }
                 const uint32_t off = umma::kstep_offset(row, 16 * hf + 4 * t);
                 *reinterpret_cast<uint2 *>(stage + (2 * d) * LEV_BYTES + off) = make_uint2(h01, h23);
-                *reinterpret_cast<uint2 *>(stage + (2 * d + 1) * LEV_BYTES + off) = make_uint2(l01, l23);
+                if (d == 0) { // the low part: level 1 only (see the header)
+                    uint32_t l01, l23;
+                    lookup4<false>(tb[d] + 8, sel, l01, l23);
+                    *reinterpret_cast<uint2 *>(stage + LEV_BYTES + off) = make_uint2(l01, l23);
+                }
             }
         }
     }
@@ -467,8 +469,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_gemm_kernel(Args a)
                                 const uint32_t dcol = acc0 + (uint32_t)(d * npad);
                                 umma::mma_f16(dcol, umma::smem_desc(S.A[st] + (2 * d) * LEV_BYTES + kh * 256), bd, idesc,
                                               !(g_first && kh == 0));
-                                umma::mma_f16(dcol, umma::smem_desc(S.A[st] + (2 * d + 1) * LEV_BYTES + kh * 256), bd,
-                                              idesc, true);
+                                if (d == 0)
+                                    umma::mma_f16(dcol, umma::smem_desc(S.A[st] + LEV_BYTES + kh * 256), bd, idesc, true);
                             }
                         umma::commit(&S.aempty[st]);
                         if (kk == KS_CH - 1)
@@ -519,9 +521,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_gemm_kernel(Args a)
 #pragma unroll
             for (int c = 0; c < kTcMaxCols; ++c)
                 R[c] = 0.0f;
+            float sg_next = __ldg(srow); // the next group's scale is loaded while a group is waited for
             for (int g = 0; g < ngr; ++g, ++gg) {
                 const int buf = gg & 1;
-                const float sg = __ldg(srow + g);
+                const float sg = sg_next;
+                if (g + 1 < ngr)
+                    sg_next = __ldg(srow + g + 1);
                 if (!pipe::mbar_wait(&S.gfull[buf], (gg >> 1) & 1, deadline)) {
                     ok = false;
                     break;
@@ -531,20 +536,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_gemm_kernel(Args a)
 #pragma unroll
                 for (int cb0 = 0; cb0 < kTcMaxCols; cb0 += 16) {
                     if (cb0 < n) {
-                        float sum[16], v[16];
-                        umma::ld16(tl + (uint32_t)cb0, sum); // level 1: every column
+                        // the four levels' 16 columns in one load (levels past the unit's depth, or past
+                        // a column's depth, are not added)
+                        float v[kTcMaxLevels][16];
+                        umma::ld16x4(tl + (uint32_t)cb0, (uint32_t)npad, v);
 #pragma unroll
-                        for (int d = 1; d < kTcMaxLevels; ++d) {
-                            if (d < nl && cb0 < nd[d]) {
-                                umma::ld16(tl + (uint32_t)(d * npad + cb0), v);
+                        for (int cc = 0; cc < 16; ++cc) {
+                            float sum = v[0][cc];
 #pragma unroll
-                                for (int cc = 0; cc < 16; ++cc)
-                                    sum[cc] += (cb0 + cc < nd[d]) ? v[cc] : 0.0f;
-                            }
+                            for (int d = 1; d < kTcMaxLevels; ++d)
+                                sum += (d < nl && cb0 + cc < nd[d]) ? v[d][cc] : 0.0f;
+                            R[cb0 + cc] = __fmaf_rn(sum, sg, R[cb0 + cc]);
                         }
-#pragma unroll
-                        for (int cc = 0; cc < 16; ++cc)
-                            R[cb0 + cc] = __fmaf_rn(sum[cc], sg, R[cb0 + cc]);
                     }
                 }
                 umma::fence_before_sync();

@@ -312,10 +312,20 @@ PMOE_API pmoe_status pmoe_moe_layer_fwd_noalloc(const pmoe_layer *L, const uint1
                                                 pmoe_stream stream);
 
 /*
+ * pmoe_set_tc_min_tokens: pairs at depth <= 4 that an expert needs in one
+ * layer call (of T >= 8 tokens) before its tensor-core units take them
+ * (process-wide; default 8). n >= 8 sets it, 0 sends every pair to the
+ * persistent kernel; INVALID_ARG for 1..7 (the workspace is sized for units
+ * of at least 8 pairs).
+ */
+PMOE_API pmoe_status pmoe_set_tc_min_tokens(int n);
+
+/*
  * pmoe_layer_counts: how the last layer call that used workspace ws grouped
  * its pairs (synchronises the stream): counts[0] column blocks and counts[1]
  * expert units of the persistent kernel, counts[2] tensor-core units (experts
- * hit by at least 8 pairs at depth <= 4, batches of T >= 8 tokens), counts[3]
+ * hit by at least 8 pairs at depth <= 4, see pmoe_set_tc_min_tokens; batches
+ * of T >= 8 tokens), counts[3]
  * their operand rows (pairs padded to multiples of 16 per unit).
  */
 PMOE_API pmoe_status pmoe_layer_counts(const void *ws, int *counts, pmoe_stream stream);
