@@ -57,12 +57,13 @@ constexpr int NDEC = 8, W_EPI = 8, NEPI = 4, W_PROD = 12, W_MMA = 13;
 constexpr int NTHREADS = 14 * 32;
 constexpr int KCH = 128;                                     // k per ring chunk (one plane tile)
 constexpr int KS_CH = KCH / 32;                              // k-steps per chunk
-constexpr int NSLOT = 2, NST = 2;                            // ring slots, decoded stages
+constexpr int NSLOT = 3, NST = 4;                            // ring slots, decoded stages
 constexpr int PLANES_CH = NDEC * kTcMaxLevels * 256;         // plane tiles of a chunk (8 KB)
 constexpr int BOPS_CH = KS_CH * kTcMaxCols * 64;             // B operand of a chunk (8 KB)
 constexpr int SLOT_BYTES = PLANES_CH + BOPS_CH;
 constexpr int LEV_BYTES = 128 * 32 * 2;                      // one level part of a decoded k-step
-constexpr int STAGE_BYTES = kTcMaxLevels * 2 * LEV_BYTES;    // levels x (high, low parts)
+constexpr int LO1 = kTcMaxLevels;                            // part index of level 1's low part
+constexpr int STAGE_BYTES = (kTcMaxLevels + 1) * LEV_BYTES;  // levels' high parts, level 1's low part
 constexpr uint64_t kDrainNs = 200ull * 1000 * 1000;
 
 struct Smem {
@@ -247,7 +248,9 @@ __device__ __forceinline__ void decode_kstep(const uint32_t (&w)[kTcMaxLevels][2
         uint32_t acc = 0;
 #pragma unroll
         for (int d = 0; d < NL; ++d) {
-            acc |= w[d][h] & dev::rotl_c(0x11111111u << d, r);
+            // (select, not an index: s is a run-time loop variable, and an indexed w would live in local
+            // memory)
+            acc |= (h ? w[d][1] : w[d][0]) & dev::rotl_c(0x11111111u << d, r);
             const uint32_t tw = r ? __funnelshift_r(acc, acc, r) : acc;
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
@@ -258,11 +261,11 @@ __device__ __forceinline__ void decode_kstep(const uint32_t (&w)[kTcMaxLevels][2
                 else
                     lookup4<false>(tb[d], sel, h01, h23);
                 const uint32_t off = umma::kstep_offset(row, 16 * hf + 4 * t);
-                *reinterpret_cast<uint2 *>(stage + (2 * d) * LEV_BYTES + off) = make_uint2(h01, h23);
+                *reinterpret_cast<uint2 *>(stage + d * LEV_BYTES + off) = make_uint2(h01, h23);
                 if (d == 0) { // the low part: level 1 only (see the header)
                     uint32_t l01, l23;
                     lookup4<false>(tb[d] + 8, sel, l01, l23);
-                    *reinterpret_cast<uint2 *>(stage + LEV_BYTES + off) = make_uint2(l01, l23);
+                    *reinterpret_cast<uint2 *>(stage + LO1 * LEV_BYTES + off) = make_uint2(l01, l23);
                 }
             }
         }
@@ -467,10 +470,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_gemm_kernel(Args a)
                             for (int kh = 0; kh < 2; ++kh) {
                                 const uint64_t bd = umma::smem_desc(bk + kh * 256);
                                 const uint32_t dcol = acc0 + (uint32_t)(d * npad);
-                                umma::mma_f16(dcol, umma::smem_desc(S.A[st] + (2 * d) * LEV_BYTES + kh * 256), bd, idesc,
+                                umma::mma_f16(dcol, umma::smem_desc(S.A[st] + d * LEV_BYTES + kh * 256), bd, idesc,
                                               !(g_first && kh == 0));
                                 if (d == 0)
-                                    umma::mma_f16(dcol, umma::smem_desc(S.A[st] + LEV_BYTES + kh * 256), bd, idesc, true);
+                                    umma::mma_f16(dcol, umma::smem_desc(S.A[st] + LO1 * LEV_BYTES + kh * 256), bd, idesc,
+                                                  true);
                             }
                         umma::commit(&S.aempty[st]);
                         if (kk == KS_CH - 1)
@@ -505,17 +509,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_gemm_kernel(Args a)
             const int grow = it.tile * 128 + row; // row of the matrix's output
             const float *srow = L.scales + (int64_t)it.e * escale_len +
                                 (MODE == 0 ? (int64_t)it.m * I * (H / G) : 2 * (int64_t)I * (H / G)) + (int64_t)grow * ngr;
-            // columns are ordered by depth, deepest first: column c takes level d iff c < nd[d]
-            int nd[kTcMaxLevels];
+            // columns are ordered by depth, deepest first: column c takes level d + 1 iff c < nd_d (the
+            // number of the unit's pairs deeper than d); held as scalars, not an array, so that they stay
+            // in registers
+            int nd1 = 0, nd2 = 0, nd3 = 0;
+            for (int c = lane; c < n; c += 32) {
+                const int dp = __ldg(W.tc_rdep + it.rowoff + c);
+                nd1 += dp > 1 ? 1 : 0;
+                nd2 += dp > 2 ? 1 : 0;
+                nd3 += dp > 3 ? 1 : 0;
+            }
 #pragma unroll
-            for (int d = 0; d < kTcMaxLevels; ++d) {
-                int cnt = 0;
-                for (int c = lane; c < n; c += 32)
-                    cnt += __ldg(W.tc_rdep + it.rowoff + c) > d ? 1 : 0;
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1)
-                    cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-                nd[d] = cnt;
+            for (int o = 16; o > 0; o >>= 1) {
+                nd1 += __shfl_xor_sync(0xffffffffu, nd1, o);
+                nd2 += __shfl_xor_sync(0xffffffffu, nd2, o);
+                nd3 += __shfl_xor_sync(0xffffffffu, nd3, o);
             }
             float R[kTcMaxCols];
 #pragma unroll
@@ -542,11 +550,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_gemm_kernel(Args a)
                         umma::ld16x4(tl + (uint32_t)cb0, (uint32_t)npad, v);
 #pragma unroll
                         for (int cc = 0; cc < 16; ++cc) {
+                            const int c = cb0 + cc;
                             float sum = v[0][cc];
-#pragma unroll
-                            for (int d = 1; d < kTcMaxLevels; ++d)
-                                sum += (d < nl && cb0 + cc < nd[d]) ? v[d][cc] : 0.0f;
-                            R[cb0 + cc] = __fmaf_rn(sum, sg, R[cb0 + cc]);
+                            sum += c < nd1 ? v[1][cc] : 0.0f; // (nd_d = 0 past the unit's depth)
+                            sum += c < nd2 ? v[2][cc] : 0.0f;
+                            sum += c < nd3 ? v[3][cc] : 0.0f;
+                            R[c] = __fmaf_rn(sum, sg, R[c]);
                         }
                     }
                 }
@@ -622,6 +631,32 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_gemm_kernel(Args a)
 // One warp per operand row (a unit's token, or a padding row): the row's values times 2^f (f: the row's
 // power-of-two scale, max |value| * 2^f in [2^13, 2^14)) as f16, in the k-step layout, for all K/32
 // k-steps; padding rows are zero. MODE 0: x (bf16) of the pair's token; MODE 1: h = silu(g) * u.
+// A lane handles 8 consecutive values at a time (two 8-byte loads of x, or four 16-byte loads of g, u).
+template <int MODE>
+__device__ __forceinline__ void row_values8(const uint16_t *__restrict__ x, const LayerWs &W, int pair, int k, int K,
+                                            int j, float (&v)[8])
+{
+    if (MODE == 0) {
+        const uint2 *p = reinterpret_cast<const uint2 *>(x + (int64_t)(pair / k) * K + j);
+        const uint2 a = __ldg(p), b = __ldg(p + 1);
+        const uint32_t w[4] = {a.x, a.y, b.x, b.y};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            v[2 * e] = __uint_as_float(w[e] << 16);
+            v[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+        }
+    } else {
+        const float4 *g = reinterpret_cast<const float4 *>(W.tc_gu + (int64_t)pair * 2 * K + j);
+        const float4 *u = reinterpret_cast<const float4 *>(W.tc_gu + (int64_t)pair * 2 * K + K + j);
+        const float4 g0 = __ldcg(g), g1 = __ldcg(g + 1), u0 = __ldcg(u), u1 = __ldcg(u + 1);
+        const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+        const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            v[e] = gv[e] / (1.0f + expf(-gv[e])) * uv[e];
+    }
+}
+
 template <int MODE>
 __global__ void tc_operand_kernel(const uint16_t *__restrict__ x, int k, int K, LayerWs W)
 {
@@ -633,45 +668,36 @@ __global__ void tc_operand_kernel(const uint16_t *__restrict__ x, int k, int K, 
     const int4 ur = W.tc_unit[W.tc_runit[gw]];
     const int npad = ur.z & 0xffff, rowoff = ur.w, r = gw - rowoff;
     unsigned char *dst = reinterpret_cast<unsigned char *>(MODE == 0 ? W.tc_xb : W.tc_hb) + (int64_t)rowoff * K * 2;
-    // value j of the row
-    auto value = [&](int j) -> float {
-        if (MODE == 0) {
-            const uint16_t b = __ldg(x + (int64_t)(pair / k) * K + j);
-            return __uint_as_float((uint32_t)b << 16);
-        } else {
-            const float g = __ldcg(W.tc_gu + (int64_t)pair * 2 * K + j);
-            const float u = __ldcg(W.tc_gu + (int64_t)pair * 2 * K + K + j);
-            return g / (1.0f + expf(-g)) * u;
-        }
-    };
     int f = 0;
     if (pair >= 0) {
         float m = 0.0f;
-        for (int j = lane; j < K; j += 32)
-            m = fmaxf(m, fabsf(value(j)));
+        for (int j = 8 * lane; j < K; j += 256) {
+            float v[8];
+            row_values8<MODE>(x, W, pair, k, K, j, v);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                m = fmaxf(m, fabsf(v[e]));
+        }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1)
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         f = pow2_exponent(m, 13);
     }
-    // lane: k-step ks (lane, lane + 32, ...), its four 8-element groups
-    for (int ks = lane; ks < K / 32; ks += 32) {
+    // lane: 8-value group g8 of k-step ks (consecutive lanes take consecutive groups)
+    for (int j = 8 * lane; j < K; j += 256) {
+        const int ks = j / 32, g8 = (j % 32) / 8;
+        float v[8];
+        if (pair >= 0)
+            row_values8<MODE>(x, W, pair, k, K, j, v);
+        uint32_t wv[4];
 #pragma unroll
-        for (int g8 = 0; g8 < 4; ++g8) {
-            uint32_t wv[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                float a0 = 0.0f, a1 = 0.0f;
-                if (pair >= 0) {
-                    a0 = ldexpf(value(ks * 32 + g8 * 8 + 2 * e), f);
-                    a1 = ldexpf(value(ks * 32 + g8 * 8 + 2 * e + 1), f);
-                }
-                const __half2 h2 = __floats2half2_rn(a0, a1);
-                wv[e] = *reinterpret_cast<const uint32_t *>(&h2);
-            }
-            *reinterpret_cast<uint4 *>(dst + (int64_t)ks * npad * 64 + umma::kstep_offset(r, g8 * 8)) =
-                make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        for (int e = 0; e < 4; ++e) {
+            const __half2 h2 = pair >= 0 ? __floats2half2_rn(ldexpf(v[2 * e], f), ldexpf(v[2 * e + 1], f))
+                                         : __floats2half2_rn(0.0f, 0.0f);
+            wv[e] = *reinterpret_cast<const uint32_t *>(&h2);
         }
+        *reinterpret_cast<uint4 *>(dst + (int64_t)ks * npad * 64 + umma::kstep_offset(r, g8 * 8)) =
+            make_uint4(wv[0], wv[1], wv[2], wv[3]);
     }
     if (lane == 0)
         (MODE == 0 ? W.tc_rxe : W.tc_rhe)[gw] = f;
