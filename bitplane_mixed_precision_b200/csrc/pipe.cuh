@@ -80,6 +80,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
     }
 }
 
+// The same without sleeping between tests: for hand-overs on a pipeline's critical path (a k-step
+// between decoding warps and the MMA thread), where a sleep adds its whole length to the latency;
+// the test itself may suspend the thread until the phase completes.
+__device__ __forceinline__ bool mbar_wait_tight(uint64_t *bar, uint32_t parity, uint64_t deadline)
+{
+    for (int it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if ((it & 15) == 0 && globaltimer() > deadline)
+            return false;
+    }
+}
+
 // Bulk copy global -> shared (this CTA), completion counted on bar in bytes.
 // dst, src 16-byte aligned; bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar)

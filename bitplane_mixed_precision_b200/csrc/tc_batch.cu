@@ -33,8 +33,9 @@
 // tc_gemm_kernel is persistent (one CTA per SM) with warp roles:
 //  * warps 0-7, decoders: warp w decodes rows 16w..16w+15 of the tile, one
 //    k-step (32 k) at a time, every level, into a shared-memory stage;
-//  * warp 12, producer: 1-D bulk copies of each 128-k chunk (the tile's planes
-//    and the unit's B operand) into a two-slot ring;
+//  * warp 12, producer: 1-D bulk copies of each chunk of up to 512 k (the
+//    tile's planes, 1 KB per plane and 16-row block, and the unit's B
+//    operand) into a two-slot ring;
 //  * warp 13: allocates tensor memory and issues the MMAs (one thread);
 //  * warps 8-11, epilogue: after each scale group, read its accumulators
 //    (tcgen05.ld), add them times the group scale into per-token fp32 sums in
@@ -55,11 +56,10 @@ namespace tc {
 
 constexpr int NDEC = 8, W_EPI = 8, NEPI = 4, W_PROD = 12, W_MMA = 13;
 constexpr int NTHREADS = 14 * 32;
-constexpr int KCH = 128;                                     // k per ring chunk (one plane tile)
-constexpr int KS_CH = KCH / 32;                              // k-steps per chunk
-constexpr int NSLOT = 3, NST = 4;                            // ring slots, decoded stages
-constexpr int PLANES_CH = NDEC * kTcMaxLevels * 256;         // plane tiles of a chunk (8 KB)
-constexpr int BOPS_CH = KS_CH * kTcMaxCols * 64;             // B operand of a chunk (8 KB)
+constexpr int TPC_MAX = 4;                                   // plane tiles (128 k each) per ring chunk
+constexpr int NSLOT = 2, NST = 2;                            // ring slots, decoded stages
+constexpr int PLANES_CH = NDEC * kTcMaxLevels * TPC_MAX * 256; // plane tiles of a chunk (32 KB)
+constexpr int BOPS_CH = 4 * TPC_MAX * kTcMaxCols * 64;        // B operand of a chunk (32 KB)
 constexpr int SLOT_BYTES = PLANES_CH + BOPS_CH;
 constexpr int LEV_BYTES = 128 * 32 * 2;                      // one level part of a decoded k-step
 constexpr int LO1 = kTcMaxLevels;                            // part index of level 1's low part
@@ -184,6 +184,7 @@ __device__ void build_level(const float *cb, int d, int fa, uint32_t *dst)
 
 struct Item {
     int u, m, tile, e, n, npad, nlev, rowoff, K;
+    int tpc; // plane tiles per ring chunk: the largest of 4, 2, 1 dividing K / 128
 };
 
 __device__ __forceinline__ bool get_item(const LayerWs &W, int mode, int idx, int H, int I, Item &o)
@@ -209,6 +210,8 @@ __device__ __forceinline__ bool get_item(const LayerWs &W, int mode, int idx, in
     o.npad = ur.z & 0xffff;
     o.nlev = ur.z >> 16;
     o.rowoff = ur.w;
+    const int nt = o.K / 128;
+    o.tpc = nt % 4 == 0 ? 4 : (nt % 2 == 0 ? 2 : 1);
     return true;
 }
 
@@ -260,7 +263,7 @@ __device__ __forceinline__ void decode_kstep(const uint32_t (&w)[kTcMaxLevels][2
                     lookup4<true>(tb[d], sel, h01, h23);
                 else
                     lookup4<false>(tb[d], sel, h01, h23);
-                const uint32_t off = umma::kstep_offset(row, 16 * hf + 4 * t);
+                const uint32_t off = umma::a_offset_sw32(row, 16 * hf + 4 * t);
                 *reinterpret_cast<uint2 *>(stage + d * LEV_BYTES + off) = make_uint2(h01, h23);
                 if (d == 0) { // the low part: level 1 only (see the header)
                     uint32_t l01, l23;
@@ -339,8 +342,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_gemm_kernel(Args a)
         int gch = 0;
         bool ok = true;
         for (int idx = blockIdx.x; ok && get_item(W, MODE, idx, H, I, it); idx += gridDim.x) {
-            const int K = it.K, nch = K / KCH;
-            const uint32_t bbytes = (uint32_t)(KS_CH * it.npad * 64);
+            const int K = it.K, tpc = it.tpc, nch = K / (128 * tpc);
+            const uint32_t bbytes = (uint32_t)(4 * tpc * it.npad * 64), pbytes = (uint32_t)(tpc * 256);
             const char *bunit = bsrc + (int64_t)it.rowoff * K * 2;
             // lane = plane p (lane / 8) and 16-row block rb (lane % 8) of the tile
             const int p = lane >> 3, rb = lane & 7;
@@ -351,18 +354,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_gemm_kernel(Args a)
             for (int c = 0; ok && c < nch; ++c, ++gch) {
                 const int slot = gch % NSLOT;
                 if (lane == 0) {
-                    if (gch >= NSLOT && !pipe::mbar_wait(&S.cempty[slot], ((gch - NSLOT) / NSLOT) & 1, deadline))
+                    if (gch >= NSLOT && !pipe::mbar_wait_tight(&S.cempty[slot], ((gch - NSLOT) / NSLOT) & 1, deadline))
                         ok = false;
                     if (ok)
-                        pipe::mbar_arrive_expect_tx(&S.full[slot], (uint32_t)__popc(have) * 256u + bbytes);
+                        pipe::mbar_arrive_expect_tx(&S.full[slot], (uint32_t)__popc(have) * pbytes + bbytes);
                 }
                 ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
                 if (!ok)
                     break;
                 if (ps >= 0) {
-                    const uint32_t *src =
-                        L.pool + (int64_t)ps * L.slot_words + it.m * mat_words + ((int64_t)(it.tile * 8 + rb) * (K / 128) + c) * 64;
-                    pipe::bulk_g2s(S.ring[slot] + (p * 8 + rb) * 256, src, 256, &S.full[slot]);
+                    const uint32_t *src = L.pool + (int64_t)ps * L.slot_words + it.m * mat_words +
+                                          ((int64_t)(it.tile * 8 + rb) * (K / 128) + c * tpc) * 64;
+                    pipe::bulk_g2s(S.ring[slot] + (p * 8 + rb) * (TPC_MAX * 256), src, pbytes, &S.full[slot]);
                 }
                 if (lane == 31)
                     pipe::bulk_g2s(S.ring[slot] + PLANES_CH, bunit + (int64_t)c * bbytes, bbytes, &S.full[slot]);
@@ -396,7 +399,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_gemm_kernel(Args a)
                 if (lane == 0)
                     pipe::mbar_arrive(&S.tabready[par]);
             }
-            if (!pipe::mbar_wait(&S.tabready[par], (n_it >> 1) & 1, deadline)) {
+            if (!pipe::mbar_wait_tight(&S.tabready[par], (n_it >> 1) & 1, deadline)) {
                 ok = false;
                 break;
             }
@@ -406,27 +409,30 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_gemm_kernel(Args a)
 #pragma unroll
                 for (int r = 0; r < 16; ++r)
                     tb[d][r] = S.tab[par][d][r];
-            const int nch = K / KCH;
+            const int tpc = it.tpc, nch = K / (128 * tpc);
             for (int c = 0; ok && c < nch; ++c, ++gch) {
                 const int slot = gch % NSLOT;
-                if (!pipe::mbar_wait(&S.full[slot], (gch / NSLOT) & 1, deadline)) {
+                if (!pipe::mbar_wait_tight(&S.full[slot], (gch / NSLOT) & 1, deadline)) {
                     ok = false;
                     break;
                 }
+#pragma unroll 1
+                for (int j = 0; ok && j < tpc; ++j) {
                 uint32_t w[kTcMaxLevels][2];
 #pragma unroll
                 for (int d = 0; d < kTcMaxLevels; ++d) {
                     w[d][0] = w[d][1] = 0u;
                     if (d < nl) {
-                        const uint2 v = *reinterpret_cast<const uint2 *>(S.ring[slot] + (d * 8 + rb) * 256 + lane * 8);
+                        const uint2 v = *reinterpret_cast<const uint2 *>(S.ring[slot] + (d * 8 + rb) * (TPC_MAX * 256) +
+                                                                           j * 256 + lane * 8);
                         w[d][0] = v.x;
                         w[d][1] = v.y;
                     }
                 }
 #pragma unroll 1
-                for (int s = 0; s < KS_CH; ++s, ++gks) {
+                for (int s = 0; s < 4; ++s, ++gks) {
                     const int st = gks % NST;
-                    if (gks >= NST && !pipe::mbar_wait(&S.aempty[st], ((gks - NST) / NST) & 1, deadline)) {
+                    if (gks >= NST && !pipe::mbar_wait_tight(&S.aempty[st], ((gks - NST) / NST) & 1, deadline)) {
                         ok = false;
                         break;
                     }
@@ -435,6 +441,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_gemm_kernel(Args a)
                     __syncwarp();
                     if (lane == 0)
                         pipe::mbar_arrive(&S.afull[st]);
+                }
                 }
             }
         }
@@ -445,21 +452,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_gemm_kernel(Args a)
         int gch = 0, gks = 0, gg = 0; // chunks, k-steps, scale groups so far
         bool ok = true;
         for (int idx = blockIdx.x; ok && get_item(W, MODE, idx, H, I, it); idx += gridDim.x) {
-            const int nch = it.K / KCH, nl = it.nlev, npad = it.npad;
+            const int ksch = 4 * it.tpc, nch = it.K / (32 * ksch), nl = it.nlev, npad = it.npad;
             const uint32_t idesc = umma::idesc_f16(128, npad);
             int ks_item = 0;
             for (int c = 0; ok && c < nch; ++c, ++gch) {
                 const int slot = gch % NSLOT;
-                if (lane == 0 && !pipe::mbar_wait(&S.full[slot], (gch / NSLOT) & 1, deadline))
+                if (lane == 0 && !pipe::mbar_wait_tight(&S.full[slot], (gch / NSLOT) & 1, deadline))
                     ok = false;
-                for (int kk = 0; ok && kk < KS_CH; ++kk, ++gks, ++ks_item) {
+                for (int kk = 0; ok && kk < ksch; ++kk, ++gks, ++ks_item) {
                     const int st = gks % NST;
                     const bool g_first = ks_item % KPG == 0, g_last = ks_item % KPG == KPG - 1;
                     const int buf = gg & 1;
                     // a group's buffer is free once the epilogue has read the group two back
-                    if (lane == 0 && g_first && gg >= 2 && !pipe::mbar_wait(&S.gempty[buf], ((gg - 2) >> 1) & 1, deadline))
+                    if (lane == 0 && g_first && gg >= 2 && !pipe::mbar_wait_tight(&S.gempty[buf], ((gg - 2) >> 1) & 1, deadline))
                         ok = false;
-                    if (lane == 0 && ok && !pipe::mbar_wait(&S.afull[st], (gks / NST) & 1, deadline))
+                    if (lane == 0 && ok && !pipe::mbar_wait_tight(&S.afull[st], (gks / NST) & 1, deadline))
                         ok = false;
                     if (lane == 0 && ok) {
                         umma::fence_after_sync();
@@ -470,14 +477,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_gemm_kernel(Args a)
                             for (int kh = 0; kh < 2; ++kh) {
                                 const uint64_t bd = umma::smem_desc(bk + kh * 256);
                                 const uint32_t dcol = acc0 + (uint32_t)(d * npad);
-                                umma::mma_f16(dcol, umma::smem_desc(S.A[st] + d * LEV_BYTES + kh * 256), bd, idesc,
+                                umma::mma_f16(dcol, umma::smem_desc_sw32(S.A[st] + d * LEV_BYTES + kh * 4096), bd, idesc,
                                               !(g_first && kh == 0));
                                 if (d == 0)
-                                    umma::mma_f16(dcol, umma::smem_desc(S.A[st] + LO1 * LEV_BYTES + kh * 256), bd, idesc,
-                                                  true);
+                                    umma::mma_f16(dcol, umma::smem_desc_sw32(S.A[st] + LO1 * LEV_BYTES + kh * 4096), bd,
+                                                  idesc, true);
                             }
                         umma::commit(&S.aempty[st]);
-                        if (kk == KS_CH - 1)
+                        if (kk == ksch - 1)
                             umma::commit(&S.cempty[slot]);
                         if (g_last)
                             umma::commit(&S.gfull[buf]);
@@ -535,7 +542,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_gemm_kernel(Args a)
                 const float sg = sg_next;
                 if (g + 1 < ngr)
                     sg_next = __ldg(srow + g + 1);
-                if (!pipe::mbar_wait(&S.gfull[buf], (gg >> 1) & 1, deadline)) {
+                if (!pipe::mbar_wait_tight(&S.gfull[buf], (gg >> 1) & 1, deadline)) {
                     ok = false;
                     break;
                 }
@@ -586,7 +593,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_gemm_kernel(Args a)
                 __syncwarp();
                 if (lane == 0)
                     pipe::mbar_arrive(&S.epidone[par]);
-                if (!pipe::mbar_wait(&S.epidone[par], (n_it >> 1) & 1, deadline)) {
+                if (!pipe::mbar_wait_tight(&S.epidone[par], (n_it >> 1) & 1, deadline)) {
                     ok = false;
                     break;
                 }
@@ -705,8 +712,8 @@ __global__ void tc_operand_kernel(const uint16_t *__restrict__ x, int k, int K, 
 
 // ---------------------------------------------------------------- tensor-core operand self-check
 
-// D[128 x N] = A[128 x K] * B[N x K]^T with the operand layout, descriptors, MMA, commit and tensor-memory
-// loads of the kernel above (one CTA, 128 threads; K <= 128 in k-steps of 32, N a multiple of 16 <= 64).
+// D[128 x N] = A[128 x K] * B[N x K]^T with the operand layouts (A swizzled, B not), descriptors, MMA,
+// commit and tensor-memory loads of the kernel above (one CTA, 128 threads; K <= 128 in k-steps of 32, N a multiple of 16 <= 64).
 constexpr int kCheckSmem = 4 * 8192 + 4 * 64 * 64;
 __global__ void __launch_bounds__(128) tc_selfcheck_kernel(const uint16_t *__restrict__ A,
                                                           const uint16_t *__restrict__ B, float *__restrict__ D,
@@ -721,7 +728,7 @@ __global__ void __launch_bounds__(128) tc_selfcheck_kernel(const uint16_t *__res
     for (int i = tid; i < nks * 128 * 4; i += 128) { // (k-step, row, 8-group)
         const int ks = i / 512, r = (i / 4) % 128, g8 = i % 4;
         const uint4 v = *reinterpret_cast<const uint4 *>(A + (int64_t)r * K + ks * 32 + g8 * 8);
-        *reinterpret_cast<uint4 *>(sa + ks * 8192 + umma::kstep_offset(r, g8 * 8)) = v;
+        *reinterpret_cast<uint4 *>(sa + ks * 8192 + umma::a_offset_sw32(r, g8 * 8)) = v;
     }
     for (int i = tid; i < nks * N * 4; i += 128) {
         const int ks = i / (N * 4), r = (i / 4) % N, g8 = i % 4;
@@ -744,8 +751,8 @@ __global__ void __launch_bounds__(128) tc_selfcheck_kernel(const uint16_t *__res
     if (tid == 0) {
         for (int ks = 0; ks < nks; ++ks)
             for (int kh = 0; kh < 2; ++kh)
-                umma::mma_f16(tm, umma::smem_desc(sa + ks * 8192 + kh * 256), umma::smem_desc(sb + ks * N * 64 + kh * 256),
-                              umma::idesc_f16(128, N), ks > 0 || kh > 0);
+                umma::mma_f16(tm, umma::smem_desc_sw32(sa + ks * 8192 + kh * 4096),
+                              umma::smem_desc(sb + ks * N * 64 + kh * 256), umma::idesc_f16(128, N), ks > 0 || kh > 0);
         umma::commit(&done);
     }
     __syncwarp();

@@ -38,6 +38,24 @@ __device__ __forceinline__ uint64_t smem_desc(const void *p)
            (1ull << 46);
 }
 
+// The A operand (128 rows, written by threads) uses the 32-byte-swizzled K-major layout instead: per
+// MMA K slice kh (16 elements) a 4 KB block of 128 rows x 32 bytes, row r at 32 r, its two 16-byte
+// chunks (k 0..7, 8..15 of the slice) swapped on rows with bit 2 set (address bit 4 ^= bit 7). Eight
+// lanes that store 8 bytes of 4 consecutive rows then hit 32 distinct banks per half-warp.
+__host__ __device__ constexpr uint32_t a_offset_sw32(int r, int k)
+{
+    return (uint32_t)((k / 16) * 4096 + r * 32 + ((((k % 16) / 8) ^ ((r >> 2) & 1)) << 4) + (k % 8) * 2);
+}
+
+// Descriptor of one K slice of that layout (start 256-byte aligned): leading byte offset 16 (unused by
+// swizzled K-major layouts), stride byte offset 256 (8 rows x 32 bytes), layout type 6 (32-byte swizzle).
+__device__ __forceinline__ uint64_t smem_desc_sw32(const void *p)
+{
+    const uint32_t a = pipe::smem_u32(p);
+    return (uint64_t)((a >> 4) & 0x3fffu) | (1ull << 16) | ((uint64_t)(256 >> 4) << 32) | (1ull << 46) |
+           (6ull << 61);
+}
+
 // Instruction descriptor of kind::f16: fp32 accumulator (bits 4-5 = 1), A and B
 // f16 (bits 7-9, 10-12 = 0), both K-major (bits 15, 16 = 0), N >> 3 in bits
 // 17-22, M >> 4 in bits 24-28.
