@@ -162,7 +162,7 @@ __global__ void __launch_bounds__(kPrepThreads) layer_prep_kernel(PrepArgs a)
         }
     }
     if (warp < n_rw) {
-        float *stage = reinterpret_cast<float *>(sm + 6 * P) + (int64_t)warp * E;
+        float *stage = reinterpret_cast<float *>(sm + 6 * P) + (int64_t)warp * E; // (used beyond 512 experts)
         for (int tok = warp; tok < T; tok += n_rw) {
             int id;
             float wt;
@@ -406,20 +406,24 @@ pmoe_status launch_layer(const pmoe_layer *L, const float *logits, const float *
         xfrag_kernel<<<(warps + 7) / 8, 256, 0, st>>>(x, T, L->H, W);
         PMOE_TRY(launch_status());
     }
-    // routing warps: at most one per token, one warp left for the x fragments, E floats each
+    // routing warps: at most one per token, one warp left for the x fragments; up to 512 experts a
+    // warp keeps the logits in registers, beyond that it stages them (E floats of shared memory each)
+    const bool staged_routing = L->E > 512;
     int n_rw = 0;
     if (logits != nullptr) {
         n_rw = (kPrepThreads / 32) - 1;
         n_rw = n_rw < T ? n_rw : T;
-        const int cap = (int)((32 * 1024) / ((size_t)L->E * sizeof(float)));
-        n_rw = n_rw < cap ? n_rw : cap;
+        if (staged_routing) {
+            const int cap = (int)((32 * 1024) / ((size_t)L->E * sizeof(float)));
+            n_rw = n_rw < cap ? n_rw : cap;
+        }
         n_rw = n_rw > 1 ? n_rw : 1;
     }
     // (the tensor-core epilogue reads one scale per group: at most 32 groups along K keep the
     // group accumulators' turnover below the decode rate)
     const bool tc = W.tc_unit != nullptr && g_tc_min > 0 && L->H / L->G <= 32 && L->I / L->G <= 32;
     PrepArgs pa{*L, logits, sens, x, T, k, B, ids, w, depth, frags_here ? 1 : 0, tc ? g_tc_min : 0, n_rw, W};
-    const size_t prep_smem = 6 * (size_t)P * sizeof(int) + (size_t)n_rw * L->E * sizeof(float);
+    const size_t prep_smem = 6 * (size_t)P * sizeof(int) + (staged_routing ? (size_t)n_rw * L->E * sizeof(float) : 0);
     if (prep_smem > 40 * 1024)
         PMOE_CUDA(cudaFuncSetAttribute(layer_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_smem));
     layer_prep_kernel<<<1, kPrepThreads, prep_smem, st>>>(pa);

@@ -421,7 +421,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
         s = c % NSLOT;
         if (c >= NSLOT && !prev_done && c - NSLOT >= prev_c0) {
             const int n1 = pq - 2; // the previous item (pq already counts the current one)
-            if (!pipe::mbar_wait(&S.qempty[n1 % QDEPTH], (n1 / QDEPTH) & 1, deadline)) {
+            if (!pipe::mbar_wait_tight(&S.qempty[n1 % QDEPTH], (n1 / QDEPTH) & 1, deadline)) {
                 set_error(W, kErrTimeout, 2);
                 ok = false;
             }
@@ -582,7 +582,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
         while (ok) {
             // claim only once the queue has room: an item is taken when this SM can start on it soon
             const int qs = pq % QDEPTH;
-            if (pq >= QDEPTH && !pipe::mbar_wait(&S.qempty[qs], ((pq / QDEPTH) + 1) & 1, deadline)) {
+            if (pq >= QDEPTH && !pipe::mbar_wait_tight(&S.qempty[qs], ((pq / QDEPTH) + 1) & 1, deadline)) {
                 set_error(W, kErrTimeout, 1);
                 break;
             }
@@ -612,7 +612,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
         uint32_t epi_phase = 0; // bit qs: parity of the next phase of epi[qs] (only handed-over items use it)
         for (int qi = 0;; ++qi) {
             const int qs = qi % QDEPTH;
-            if (!pipe::mbar_wait(&S.qfull[qs], (qi / QDEPTH) & 1, deadline)) {
+            if (!pipe::mbar_wait_tight(&S.qfull[qs], (qi / QDEPTH) & 1, deadline)) {
                 set_error(W, kErrTimeout, 7);
                 break;
             }
@@ -627,7 +627,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
                     pipe::mbar_arrive(&S.qempty[qs]);
                 continue;
             }
-            if (!pipe::mbar_wait(&S.epi[qs], (epi_phase >> qs) & 1u, deadline)) {
+            if (!pipe::mbar_wait_tight(&S.epi[qs], (epi_phase >> qs) & 1u, deadline)) {
                 set_error(W, kErrTimeout, 8);
                 break;
             }
@@ -689,7 +689,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
     const int g = lane >> 2, t = lane & 3;
     for (int qi = 0;; ++qi) {
         const int qs = qi % QDEPTH;
-        if (!pipe::mbar_wait(&S.qfull[qs], (qi / QDEPTH) & 1, deadline)) {
+        if (!pipe::mbar_wait_tight(&S.qfull[qs], (qi / QDEPTH) & 1, deadline)) {
             set_error(W, kErrTimeout, 3);
             break;
         }
@@ -703,7 +703,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
         bool fine = true;
         const int cm = d.c0 + bmax; // meta chunk (after the item's planes)
         const unsigned char *meta = S.ring[cm % NSLOT];
-        if (!pipe::mbar_wait(&S.ifull[qs], (qi / QDEPTH) & 1, deadline)) // the item's bytes
+        if (!pipe::mbar_wait_tight(&S.ifull[qs], (qi / QDEPTH) & 1, deadline)) // the item's bytes
             fine = false;
 
         if (d.kind == 0) {
