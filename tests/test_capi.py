@@ -82,10 +82,32 @@ def test_invalid_arguments_are_rejected_on_the_host(pm):
                          np.zeros(40, np.uint8), on_device=False)
 
 
+def test_tensor_core_settings_are_checked_on_the_host(pm):
+    """The tensor-core threshold takes 0 (off) or >= 8 (units are sized for at least 8 pairs); the
+    operand self-check refuses shapes outside N in {16, 32, 48, 64}, K in {32, 64, 96, 128} before
+    touching the device."""
+    for bad in (-1, 1, 7):
+        with pytest.raises(pm.PmoeError) as ei:
+            pm.set_tc_min_tokens(bad)
+        assert ei.value.code == 1
+    for good in (0, 8, 16, 8):
+        pm.set_tc_min_tokens(good)
+    a = np.zeros((128, 128), np.int16)
+    d = np.zeros((128, 64), np.float32)
+    for N, K in ((8, 64), (24, 64), (80, 64), (32, 16), (32, 160), (32, 48)):
+        with pytest.raises(pm.PmoeError) as ei:
+            pm.tc_selfcheck(a, a, d, N, K)
+        assert ei.value.code == 1
+
+
 def test_workspace_queries(pm):
     a = pm.layer_workspace_bytes(1, 10, 512, 4096, 1024)
     b = pm.layer_workspace_bytes(32, 10, 512, 4096, 1024)
     assert 0 < a < b
+    # batches of 8 tokens or more carry the tensor-core operand rows (3 x pairs rows of H and I
+    # halves) and the gate/up rows of tensor-core pairs
+    c7, c8 = pm.layer_workspace_bytes(7, 10, 512, 4096, 1024), pm.layer_workspace_bytes(8, 10, 512, 4096, 1024)
+    assert c8 - c7 > 80 * (4096 + 1024) * 2
     m = pm.materialise_workspace_bytes(1, 10, 512, 4096, 1024)
     assert m >= 10 * 3 * 4096 * 1024 * 2  # bf16 copies of the ten selected experts
 
