@@ -504,7 +504,7 @@ def batch_bench(args):
         per_exp.append(Tb * K_TOP / len(bmax))
     achieved = float(sum(alg) / sum(kdur)) / 1e9
     pk, pk_kind = peaks()
-    # tensor-core units of each batch (experts with >= 8 pairs at depth <= 4, units of <= 32 pairs):
+    # tensor-core units of each batch (experts with >= 8 pairs at depth <= 4, units of <= 64 pairs):
     # counted by the library, and their MMA work (2 parts x levels x 2 flop per weight and token)
     tc_units, tc_rows, tc_pairs, tc_flop = [], [], [], []
     for b in range(nb):
@@ -520,7 +520,7 @@ def batch_bench(args):
                 continue
             pairs += n
             d = np.sort(dep_h[b][sel])[::-1]
-            nun = (n + 31) // 32
+            nun = (n + 63) // 64
             for j, start in enumerate(np.cumsum([0] + [n // nun + (1 if i < n % nun else 0) for i in range(nun)])[:-1]):
                 m = n // nun + (1 if j < n % nun else 0)
                 npad = (m + 15) // 16 * 16

@@ -18,7 +18,7 @@ constexpr int kMaxMembers = 2;      // tokens per column block: 3 byte columns e
 // form units of at most kTcMaxCols pairs.
 constexpr int kTcMinTokens = 8;
 constexpr int kTcMaxLevels = 4;
-constexpr int kTcMaxCols = 32;
+constexpr int kTcMaxCols = 64;
 
 // Operand rows of the tensor-core units of a call with P pairs: every unit holds >= kTcMinTokens
 // pairs and pads them to a multiple of 16 rows.

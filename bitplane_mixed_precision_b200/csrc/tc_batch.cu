@@ -3,7 +3,7 @@
 // multiplied on the fifth-generation tensor cores (tcgen05) instead of being
 // decoded again for every pair of tokens.
 //
-// For such an expert ("TC unit": one expert, up to 32 of its (token, slot)
+// For such an expert ("TC unit": one expert, up to 64 of its (token, slot)
 // pairs, all at depth <= 4) the tree value at depth b is written as a sum of
 // level deltas (children = parent + delta):
 //     C_b[i] = sum_{d=1..b} Delta_d[i >> (b-d)],  Delta_1 = C_1,
@@ -59,7 +59,8 @@ constexpr int NTHREADS = 14 * 32;
 constexpr int TPC_MAX = 4;                                   // plane tiles (128 k each) per ring chunk
 constexpr int NSLOT = 2, NST = 2;                            // ring slots, decoded stages
 constexpr int PLANES_CH = NDEC * kTcMaxLevels * TPC_MAX * 256; // plane tiles of a chunk (32 KB)
-constexpr int BOPS_CH = 4 * TPC_MAX * kTcMaxCols * 64;        // B operand of a chunk (32 KB)
+constexpr int BOPS_CH = 32 * 1024;                           // B operand of a chunk (tiles x 4 k-steps x
+                                                             // npad x 64 B: items of 64 columns take 2 tiles)
 constexpr int SLOT_BYTES = PLANES_CH + BOPS_CH;
 constexpr int LEV_BYTES = 128 * 32 * 2;                      // one level part of a decoded k-step
 constexpr int LO1 = kTcMaxLevels;                            // part index of level 1's low part
@@ -184,7 +185,7 @@ __device__ void build_level(const float *cb, int d, int fa, uint32_t *dst)
 
 struct Item {
     int u, m, tile, e, n, npad, nlev, rowoff, K;
-    int tpc; // plane tiles per ring chunk: the largest of 4, 2, 1 dividing K / 128
+    int tpc; // plane tiles per ring chunk: the largest of 4, 2, 1 dividing K / 128 whose B operand fits
 };
 
 __device__ __forceinline__ bool get_item(const LayerWs &W, int mode, int idx, int H, int I, Item &o)
@@ -210,8 +211,8 @@ __device__ __forceinline__ bool get_item(const LayerWs &W, int mode, int idx, in
     o.npad = ur.z & 0xffff;
     o.nlev = ur.z >> 16;
     o.rowoff = ur.w;
-    const int nt = o.K / 128;
-    o.tpc = nt % 4 == 0 ? 4 : (nt % 2 == 0 ? 2 : 1);
+    const int nt = o.K / 128, cap = BOPS_CH / (4 * 64 * o.npad); // the chunk's B operand fits its region
+    o.tpc = (nt % 4 == 0 && cap >= 4) ? 4 : ((nt % 2 == 0 && cap >= 2) ? 2 : 1);
     return true;
 }
 
@@ -240,8 +241,8 @@ __device__ __forceinline__ void lookup4(const uint32_t *t, uint32_t sel, uint32_
 // d < NL: the high and low f16 parts of Delta_d * 2^fa, stored into the stage's level blocks.
 template <int NL>
 __device__ __forceinline__ void decode_kstep(const uint32_t (&w)[kTcMaxLevels][2], int s,
-                                             const uint32_t (&tb)[kTcMaxLevels][16], unsigned char *stage,
-                                             int rb, int lane)
+                                             const uint32_t (&tb)[kTcMaxLevels][8], const uint32_t (&tlo)[8],
+                                             unsigned char *stage, int rb, int lane)
 {
     const int t = lane & 3, gq = lane >> 2;
 #pragma unroll
@@ -267,7 +268,7 @@ __device__ __forceinline__ void decode_kstep(const uint32_t (&w)[kTcMaxLevels][2
                 *reinterpret_cast<uint2 *>(stage + d * LEV_BYTES + off) = make_uint2(h01, h23);
                 if (d == 0) { // the low part: level 1 only (see the header)
                     uint32_t l01, l23;
-                    lookup4<false>(tb[d] + 8, sel, l01, l23);
+                    lookup4<false>(tlo, sel, l01, l23);
                     *reinterpret_cast<uint2 *>(stage + LO1 * LEV_BYTES + off) = make_uint2(l01, l23);
                 }
             }
@@ -284,14 +285,14 @@ namespace tc {
 // ---------------------------------------------------------------- the MMA kernel
 
 __device__ __forceinline__ void decode_any(int nl, const uint32_t (&w)[kTcMaxLevels][2], int s,
-                                           const uint32_t (&tb)[kTcMaxLevels][16], unsigned char *stage, int rb,
-                                           int lane)
+                                           const uint32_t (&tb)[kTcMaxLevels][8], const uint32_t (&tlo)[8],
+                                           unsigned char *stage, int rb, int lane)
 {
     switch (nl) {
-    case 1: decode_kstep<1>(w, s, tb, stage, rb, lane); break;
-    case 2: decode_kstep<2>(w, s, tb, stage, rb, lane); break;
-    case 3: decode_kstep<3>(w, s, tb, stage, rb, lane); break;
-    default: decode_kstep<4>(w, s, tb, stage, rb, lane); break;
+    case 1: decode_kstep<1>(w, s, tb, tlo, stage, rb, lane); break;
+    case 2: decode_kstep<2>(w, s, tb, tlo, stage, rb, lane); break;
+    case 3: decode_kstep<3>(w, s, tb, tlo, stage, rb, lane); break;
+    default: decode_kstep<4>(w, s, tb, tlo, stage, rb, lane); break;
     }
 }
 
@@ -403,12 +404,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_gemm_kernel(Args a)
                 ok = false;
                 break;
             }
-            uint32_t tb[kTcMaxLevels][16];
+            uint32_t tb[kTcMaxLevels][8], tlo[8]; // high parts of every level; low part of level 1
 #pragma unroll
             for (int d = 0; d < kTcMaxLevels; ++d)
 #pragma unroll
-                for (int r = 0; r < 16; ++r)
+                for (int r = 0; r < 8; ++r)
                     tb[d][r] = S.tab[par][d][r];
+#pragma unroll
+            for (int r = 0; r < 8; ++r)
+                tlo[r] = S.tab[par][0][8 + r];
             const int tpc = it.tpc, nch = K / (128 * tpc);
             for (int c = 0; ok && c < nch; ++c, ++gch) {
                 const int slot = gch % NSLOT;
@@ -436,7 +440,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_gemm_kernel(Args a)
                         ok = false;
                         break;
                     }
-                    decode_any(nl, w, s, tb, S.A[st], rb, lane);
+                    decode_any(nl, w, s, tb, tlo, S.A[st], rb, lane);
                     umma::fence_smem_async();
                     __syncwarp();
                     if (lane == 0)
@@ -551,19 +555,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_gemm_kernel(Args a)
 #pragma unroll
                 for (int cb0 = 0; cb0 < kTcMaxCols; cb0 += 16) {
                     if (cb0 < n) {
-                        // the four levels' 16 columns in one load (levels past the unit's depth, or past
-                        // a column's depth, are not added)
-                        float v[kTcMaxLevels][16];
-                        umma::ld16x4(tl + (uint32_t)cb0, (uint32_t)npad, v);
+                        // the levels' 16 columns, two levels per load (levels past the unit's depth, or
+                        // past a column's depth, are not added: nd_d = 0 past the unit's depth)
+                        float v[2][16], sum[16];
+                        umma::ld16x2(tl + (uint32_t)cb0, (uint32_t)npad, v);
 #pragma unroll
-                        for (int cc = 0; cc < 16; ++cc) {
-                            const int c = cb0 + cc;
-                            float sum = v[0][cc];
-                            sum += c < nd1 ? v[1][cc] : 0.0f; // (nd_d = 0 past the unit's depth)
-                            sum += c < nd2 ? v[2][cc] : 0.0f;
-                            sum += c < nd3 ? v[3][cc] : 0.0f;
-                            R[c] = __fmaf_rn(sum, sg, R[c]);
+                        for (int cc = 0; cc < 16; ++cc)
+                            sum[cc] = v[0][cc] + (cb0 + cc < nd1 ? v[1][cc] : 0.0f);
+                        if (cb0 < nd2) {
+                            umma::ld16x2(tl + (uint32_t)(2 * npad + cb0), (uint32_t)npad, v);
+#pragma unroll
+                            for (int cc = 0; cc < 16; ++cc)
+                                sum[cc] += (cb0 + cc < nd2 ? v[0][cc] : 0.0f) + (cb0 + cc < nd3 ? v[1][cc] : 0.0f);
                         }
+#pragma unroll
+                        for (int cc = 0; cc < 16; ++cc)
+                            R[cb0 + cc] = __fmaf_rn(sum[cc], sg, R[cb0 + cc]);
                     }
                 }
                 umma::fence_before_sync();

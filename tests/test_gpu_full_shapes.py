@@ -112,7 +112,7 @@ def test_large_layer_zipf_batch_of_32(pm, big):
 @pytest.mark.parametrize("T", [64, 128])
 def test_large_layer_zipf_batches_of_64_and_128(pm, big, T):
     """Larger Zipf(1.1)-biased batches: the popular experts go to the tensor-core units (one
-    accumulator per tree level, up to 32 pairs each); routing and selection bit-exact, a sample of
+    accumulator per tree level, up to 64 pairs each); routing and selection bit-exact, a sample of
     tokens (those with the most tensor-core pairs and a few others) element-wise against the oracle."""
     R, O = big
     sens = synth.sensitivities(SEED, 0, E)

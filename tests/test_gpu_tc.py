@@ -5,8 +5,8 @@
 * Layers whose popular experts are hit by 8 or more pairs at depths 1..4 (they go to the tensor
   cores, one accumulator per tree level) next to deeper pairs of the same experts and rare experts
   (they stay with the persistent kernel): every token's output against the oracle's dequantise-then-
-  multiply, at the workloads' tolerance. Batches of 24 and 128 tokens; both give an expert more pairs
-  than one unit holds (32), so its pairs are split between units.
+  multiply, at the workloads' tolerance. Batches of 24 and 128 tokens; the 128-token batch gives an
+  expert more pairs than one unit holds (64), so its pairs are split between two units.
 PagedMoE transcript cues 13, 29, 35 (pairs grouped per expert, tokens at different depths sharing the
 planes they have in common).
 """
@@ -88,9 +88,9 @@ def test_layer_with_tensor_core_units(pm, mid, T):
     torch.cuda.synchronize()
     assert pm.layer_error(ws) == (0, 0)
     blocks, units, tcu, rows = pm.layer_counts(ws)
-    # every expert with at least 8 pairs at depth <= 4 gives them to units of at most 32 pairs
+    # every expert with at least 8 pairs at depth <= 4 gives them to units of at most 64 pairs
     shallow = np.bincount(ids[dep <= 4], minlength=E)
-    expect = sum((int(n) + 31) // 32 for n in shallow if n >= 8)
+    expect = sum((int(n) + 63) // 64 for n in shallow if n >= 8)
     assert tcu == expect >= 3, (tcu, expect)
     assert rows >= int(shallow[shallow >= 8].sum()) and rows % 16 == 0
     ref = O.run(E, ids, w, dep, synth.bf16_to_f32(x).astype(np.float64))
