@@ -63,6 +63,8 @@ _SIGS = {
     "pmoe_select_prefix_table": ([P, P, P, i32, i32, f32, P, i32, P], i32),
     "pmoe_expert_gemv": ([ctypes.POINTER(Matrix), i32, P, i32, P, P], i32),
     "pmoe_layer_workspace_bytes": ([i32, i32, i32, i32, i32], sz),
+    "pmoe_decode_host_workspace_bytes": ([i32, i32, i32, i32, i32], sz),
+    "pmoe_moe_decode_step_host": ([ctypes.POINTER(Layer), P, P, P, i32, i32, f32, P, P, sz, P], i32),
     "pmoe_moe_layer_fwd": ([ctypes.POINTER(Layer), P, P, P, P, i32, i32, P, P, sz, P], i32),
     "pmoe_moe_decode_step": ([ctypes.POINTER(Layer), P, P, P, i32, i32, f32, P, P, P, P, P, sz, P],
                              i32),
@@ -245,6 +247,18 @@ def moe_decode_step(L: Layer, logits, sens, x, T, k, avg_bits, y, ids_out, w_out
     _check("pmoe_moe_decode_step", _lib.pmoe_moe_decode_step(
         ctypes.byref(L), _ptr(logits), _ptr(sens), _ptr(x), T, k, avg_bits, _ptr(y), _ptr(ids_out),
         _ptr(w_out), _ptr(depth_out), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def decode_host_workspace_bytes(T, k, E, H, I) -> int:
+    return _lib.pmoe_decode_host_workspace_bytes(T, k, E, H, I)
+
+
+def moe_decode_step_host(L: Layer, logits, sens, x, T, k, avg_bits, y, ws, ws_bytes, stream=None) -> None:
+    """The decode step with logits, x and y in (pinned) host memory: one call queues the input
+    copies, the step and the output copy on the stream."""
+    _check("pmoe_moe_decode_step_host", _lib.pmoe_moe_decode_step_host(
+        ctypes.byref(L), _ptr(logits), _ptr(sens), _ptr(x), T, k, avg_bits, _ptr(y), _ptr(ws), ws_bytes,
+        _stream(stream)))
 
 
 def profile_events(start, stop) -> None:

@@ -384,6 +384,7 @@ pmoe_status check_layer(const pmoe_layer *L, int T, int k)
 }
 
 static int g_num_sms[128] = {};
+static unsigned g_smem_set[128] = {}; // per device: persistent-kernel variants whose shared-memory limit is set
 static uint64_t g_wait_limit_ns = 200ull * 1000 * 1000;
 static int g_tc_min = kTcMinTokens;
 
@@ -447,7 +448,11 @@ pmoe_status launch_layer(const pmoe_layer *L, const float *logits, const float *
     case 64: kern = mk::moe_main_kernel<2>; break;
     default: kern = mk::moe_main_kernel<4>; break;
     }
-    PMOE_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    const unsigned vbit = 1u << (L->G == 32 ? 0 : (L->G == 64 ? 1 : 2));
+    if (!(g_smem_set[dev] & vbit)) {
+        PMOE_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        g_smem_set[dev] |= vbit;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(g_num_sms[dev]);
     cfg.blockDim = dim3(mk::NTHREADS);
@@ -487,6 +492,14 @@ size_t pmoe_layer_workspace_bytes(int T, int k, int E, int H, int I)
     size_t b = 0;
     carve_layer_ws(nullptr, T, k, H, I, &b);
     return b;
+}
+
+size_t pmoe_decode_host_workspace_bytes(int T, int k, int E, int H, int I)
+{
+    const size_t b = pmoe_layer_workspace_bytes(T, k, E, H, I);
+    if (b == 0 || E <= 0)
+        return 0;
+    return b + al256((size_t)T * E * 4) + al256((size_t)T * H * 2) + al256((size_t)T * H * 4);
 }
 
 pmoe_status pmoe_set_wait_limit_ns(uint64_t ns)
@@ -564,6 +577,33 @@ pmoe_status pmoe_moe_decode_step(const pmoe_layer *L, const float *logits, const
     uint8_t *depth = depth_out ? depth_out : W.depth;
     return launch_layer(L, logits, sens, x, ids, w, depth, T, k, select_budget(k, avg_bits), y, ws, ws_bytes,
                         (cudaStream_t)stream);
+}
+
+pmoe_status pmoe_moe_decode_step_host(const pmoe_layer *L, const float *logits, const float *sens,
+                                      const uint16_t *x, int T, int k, float avg_bits, float *y, void *ws,
+                                      size_t ws_bytes, pmoe_stream stream)
+{
+    PMOE_TRY(check_layer(L, T, k));
+    if (T == 0)
+        return PMOE_OK;
+    if (!logits || !sens || !x || !y || !ws || !aligned(ws, 256))
+        return PMOE_ERR_INVALID_ARG;
+    if (ws_bytes < pmoe_decode_host_workspace_bytes(T, k, L->E, L->H, L->I))
+        return PMOE_ERR_WORKSPACE;
+    // [layer workspace | logits | x | y]: the inputs are staged next to the layer's scratch
+    const size_t lb = pmoe_layer_workspace_bytes(T, k, L->E, L->H, L->I);
+    const size_t nl = (size_t)T * L->E * 4, nx = (size_t)T * L->H * 2, ny = (size_t)T * L->H * 4;
+    char *b = static_cast<char *>(ws);
+    float *logits_d = reinterpret_cast<float *>(b + lb);
+    uint16_t *x_d = reinterpret_cast<uint16_t *>(b + lb + al256(nl));
+    float *y_d = reinterpret_cast<float *>(b + lb + al256(nl) + al256(nx));
+    const cudaStream_t st = (cudaStream_t)stream;
+    PMOE_CUDA(cudaMemcpyAsync(logits_d, logits, nl, cudaMemcpyHostToDevice, st));
+    PMOE_CUDA(cudaMemcpyAsync(x_d, x, nx, cudaMemcpyHostToDevice, st));
+    PMOE_TRY(pmoe_moe_decode_step(L, logits_d, sens, x_d, T, k, avg_bits, y_d, nullptr, nullptr, nullptr, ws, lb,
+                                  stream));
+    PMOE_CUDA(cudaMemcpyAsync(y, y_d, ny, cudaMemcpyDeviceToHost, st));
+    return PMOE_OK;
 }
 
 } // extern "C"

@@ -376,6 +376,26 @@ PMOE_API pmoe_status pmoe_moe_decode_step(const pmoe_layer *L, const float *logi
                                  size_t ws_bytes, pmoe_stream stream);
 
 /*
+ * pmoe_moe_decode_step_host: pmoe_moe_decode_step for tokens whose inputs and
+ * output live in host memory, as a serving loop holds them: copies logits
+ * (host float [T*E]) and x (host bf16 [T*H]) into the workspace, runs the
+ * step there and copies y (host float [T*H]) back, all queued on `stream` in
+ * this one call (the routing and depths stay in the workspace). The call
+ * returns once the work is queued: y is written when the stream reaches it.
+ * Page-locked (pinned) host buffers keep the copies asynchronous; pageable
+ * ones are accepted and make the copies synchronise with the host.
+ *   sens: device float [E]. ws: device scratch of >=
+ *   pmoe_decode_host_workspace_bytes() bytes, 256-byte aligned (smaller:
+ *   PMOE_ERR_WORKSPACE). Shapes and errors as pmoe_moe_decode_step.
+ */
+PMOE_API pmoe_status pmoe_moe_decode_step_host(const pmoe_layer *L, const float *logits, const float *sens,
+                                      const uint16_t *x, int T, int k, float avg_bits, float *y, void *ws,
+                                      size_t ws_bytes, pmoe_stream stream);
+
+/* Workspace of pmoe_moe_decode_step_host: the layer workspace plus room for T tokens' logits, x and y. */
+PMOE_API size_t pmoe_decode_host_workspace_bytes(int T, int k, int E, int H, int I);
+
+/*
  * pmoe_profile_events: when both events are non-NULL, every later
  * pmoe_moe_layer_fwd / pmoe_moe_decode_step call on this host thread records
  * `start` on its stream just before the expert kernels (gate/up + SwiGLU and

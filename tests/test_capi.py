@@ -112,6 +112,30 @@ def test_workspace_queries(pm):
     assert m >= 10 * 3 * 4096 * 1024 * 2  # bf16 copies of the ten selected experts
 
 
+def test_host_buffer_decode_step_is_checked_on_the_host(pm):
+    """The host-buffer decode step's workspace is the layer workspace plus 256-byte-padded room for
+    the tokens' logits, x and y; null buffers and a short workspace are refused before any copy
+    (the layer record only has to look valid: nothing is read from it on these paths)."""
+    T, k, E, H, I = 3, 10, 512, 4096, 1024
+    al = lambda n: (n + 255) // 256 * 256
+    lb = pm.layer_workspace_bytes(T, k, E, H, I)
+    assert pm.decode_host_workspace_bytes(T, k, E, H, I) == lb + al(T * E * 4) + al(T * H * 2) + al(T * H * 4)
+    assert pm.decode_host_workspace_bytes(T, 0, E, H, I) == 0
+    L = pm.Layer(E=E, H=H, I=I, G=128, pool=0x100000, slot_words=3 * H * I // 32, slot_of=0x200000,
+                 scales=0x300000, codebooks=0x400000)
+    host = np.zeros(T * H, np.float32)
+    need = pm.decode_host_workspace_bytes(T, k, E, H, I)
+    args = dict(logits=host, sens=0x500000, x=host, y=host, ws=0x600000)
+    for missing in ("logits", "sens", "x", "y", "ws"):
+        a = dict(args, **{missing: None})
+        with pytest.raises(pm.PmoeError) as ei:
+            pm.moe_decode_step_host(L, a["logits"], a["sens"], a["x"], T, k, 2.5, a["y"], a["ws"], need)
+        assert ei.value.code == 1, missing
+    with pytest.raises(pm.PmoeError) as ei:
+        pm.moe_decode_step_host(L, host, 0x500000, host, T, k, 2.5, host, 0x600000, need - 256)
+    assert ei.value.code == 5
+
+
 def test_cache_aware_select_matches_oracle(pm, oracle_mod):
     rng = np.random.default_rng(11)
     T, k, E = 64, 10, 512
