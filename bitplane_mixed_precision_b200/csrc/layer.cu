@@ -494,6 +494,25 @@ size_t pmoe_layer_workspace_bytes(int T, int k, int E, int H, int I)
     return b;
 }
 
+} // extern "C"
+
+// Device address of page-locked host memory that is mapped into the current device's address
+// space (the CUDA runtime's attributes of the pointer), else nullptr: pageable memory, device
+// memory, or pinned memory registered without a mapping.
+static void *mapped_host(const void *p)
+{
+    cudaPointerAttributes at{};
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        (void)cudaGetLastError(); // (older runtimes report pageable memory as an error)
+        return nullptr;
+    }
+    if (at.type != cudaMemoryTypeHost || at.devicePointer == nullptr)
+        return nullptr;
+    return at.devicePointer;
+}
+
+extern "C" {
+
 size_t pmoe_decode_host_workspace_bytes(int T, int k, int E, int H, int I)
 {
     const size_t b = pmoe_layer_workspace_bytes(T, k, E, H, I);
@@ -590,19 +609,33 @@ pmoe_status pmoe_moe_decode_step_host(const pmoe_layer *L, const float *logits, 
         return PMOE_ERR_INVALID_ARG;
     if (ws_bytes < pmoe_decode_host_workspace_bytes(T, k, L->E, L->H, L->I))
         return PMOE_ERR_WORKSPACE;
-    // [layer workspace | logits | x | y]: the inputs are staged next to the layer's scratch
+    // Page-locked host buffers mapped into the device's address space are read and written by the
+    // kernels in place (the prep kernel reads logits and x, the combine writes y); others go
+    // through [layer workspace | logits | x | y] with copies queued on the stream.
     const size_t lb = pmoe_layer_workspace_bytes(T, k, L->E, L->H, L->I);
     const size_t nl = (size_t)T * L->E * 4, nx = (size_t)T * L->H * 2, ny = (size_t)T * L->H * 4;
     char *b = static_cast<char *>(ws);
-    float *logits_d = reinterpret_cast<float *>(b + lb);
-    uint16_t *x_d = reinterpret_cast<uint16_t *>(b + lb + al256(nl));
-    float *y_d = reinterpret_cast<float *>(b + lb + al256(nl) + al256(nx));
     const cudaStream_t st = (cudaStream_t)stream;
-    PMOE_CUDA(cudaMemcpyAsync(logits_d, logits, nl, cudaMemcpyHostToDevice, st));
-    PMOE_CUDA(cudaMemcpyAsync(x_d, x, nx, cudaMemcpyHostToDevice, st));
+    const float *logits_d = static_cast<const float *>(mapped_host(logits));
+    const uint16_t *x_d = static_cast<const uint16_t *>(mapped_host(x));
+    float *y_d = static_cast<float *>(mapped_host(y));
+    if (!logits_d) {
+        float *p = reinterpret_cast<float *>(b + lb);
+        PMOE_CUDA(cudaMemcpyAsync(p, logits, nl, cudaMemcpyHostToDevice, st));
+        logits_d = p;
+    }
+    if (!x_d || !aligned(x_d, 8)) {
+        uint16_t *p = reinterpret_cast<uint16_t *>(b + lb + al256(nl));
+        PMOE_CUDA(cudaMemcpyAsync(p, x, nx, cudaMemcpyHostToDevice, st));
+        x_d = p;
+    }
+    const bool y_copy = y_d == nullptr;
+    if (y_copy)
+        y_d = reinterpret_cast<float *>(b + lb + al256(nl) + al256(nx));
     PMOE_TRY(pmoe_moe_decode_step(L, logits_d, sens, x_d, T, k, avg_bits, y_d, nullptr, nullptr, nullptr, ws, lb,
                                   stream));
-    PMOE_CUDA(cudaMemcpyAsync(y, y_d, ny, cudaMemcpyDeviceToHost, st));
+    if (y_copy)
+        PMOE_CUDA(cudaMemcpyAsync(y, y_d, ny, cudaMemcpyDeviceToHost, st));
     return PMOE_OK;
 }
 

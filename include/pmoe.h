@@ -382,8 +382,11 @@ PMOE_API pmoe_status pmoe_moe_decode_step(const pmoe_layer *L, const float *logi
  * step there and copies y (host float [T*H]) back, all queued on `stream` in
  * this one call (the routing and depths stay in the workspace). The call
  * returns once the work is queued: y is written when the stream reaches it.
- * Page-locked (pinned) host buffers keep the copies asynchronous; pageable
- * ones are accepted and make the copies synchronise with the host.
+ * Page-locked host buffers mapped into the device's address space (as
+ * cudaHostAlloc/cudaMallocHost memory is under unified addressing) are read
+ * and written by the kernels in place, with no copies; other page-locked
+ * buffers are copied asynchronously; pageable ones are accepted and make the
+ * copies synchronise with the host. The result is the same either way.
  *   sens: device float [E]. ws: device scratch of >=
  *   pmoe_decode_host_workspace_bytes() bytes, 256-byte aligned (smaller:
  *   PMOE_ERR_WORKSPACE). Shapes and errors as pmoe_moe_decode_step.
