@@ -514,7 +514,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_gemm_kernel(Args a)
         int gg = 0, n_it = 0;
         bool ok = true;
         for (int idx = blockIdx.x; ok && get_item(W, MODE, idx, H, I, it); idx += gridDim.x, ++n_it) {
-            const int par = n_it & 1, K = it.K, ngr = K / G, nl = it.nlev, npad = it.npad, n = it.n;
+            const int par = n_it & 1, K = it.K, ngr = K / G, npad = it.npad, n = it.n;
             const float *cb = L.codebooks + ((int64_t)it.e * 3 + it.m) * 510;
             const int fa = table_exponent(cb);
             const int grow = it.tile * 128 + row; // row of the matrix's output

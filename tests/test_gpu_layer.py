@@ -115,11 +115,13 @@ def test_group_size_64(pm):
     check_layer(pm, 42, 16, 1024, 512, 64, 4, 3)
 
 
-@pytest.mark.parametrize("T", [1, 3])
-def test_host_buffer_decode_step_matches_device_buffers(pm, T):
+@pytest.mark.parametrize("T,k", [(1, 4), (3, 4), (24, 10)])
+def test_host_buffer_decode_step_matches_device_buffers(pm, T, k):
     """pmoe_moe_decode_step_host (logits, x and y in pinned host memory, one call per step) gives
-    the device-buffer decode step's output bit for bit; pageable host buffers give it too."""
-    seed, E, H, I, G, k = 33, 16, 1024, 256, 128, 4
+    the device-buffer decode step's output bit for bit; pageable host buffers give it too. 24
+    tokens of top-10 over 16 experts put pairs on the tensor-core units, whose operand kernel then
+    reads x from the host buffer."""
+    seed, E, H, I, G = 33, 16, 1024, 256, 128
     R = ResidentLayer(E, H, I, G, device_fill(seed))
     sens = synth.sensitivities(seed, 0, E)
     logits, xb = tokens(seed, T, E, H)
@@ -134,6 +136,8 @@ def test_host_buffer_decode_step_matches_device_buffers(pm, T):
     torch.cuda.synchronize()
     assert pm.layer_error(ws) == (0, 0)
     np.testing.assert_array_equal(y.numpy().reshape(T, H), y_dev)
+    if T >= 24:
+        assert pm.layer_counts(ws)[2] > 0  # tensor-core units were formed
     y_np = np.full(T * H, np.nan, np.float32)
     pm.moe_decode_step_host(R.layer, np.ascontiguousarray(logits), d_sens, xb.view(np.int16).copy(), T, k, 2.5,
                             y_np, ws, nb)
