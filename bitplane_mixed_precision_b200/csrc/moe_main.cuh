@@ -706,193 +706,148 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_main_kernel(Args a)
         if (!pipe::mbar_wait_tight(&S.ifull[qs], (qi / QDEPTH) & 1, deadline)) // the item's bytes
             fine = false;
 
-        if (d.kind == 0) {
-            // gate/up: warp -> matrix m (warps 0-7 gate, 8-15 up) and K part kp (of 8) of the
-            // item's 16 rows; a plane chunk holds [gate rows | up rows] of one plane
-            const int m = warp >> 3, kp = warp & 7, tpw = (H / 128) / 8, Q0 = kp * tpw;
-            const int tix0 = m * (H / 128) + Q0;
-            const int ngr = H / G;
-            const unsigned char *pp[8];
+        // The warp's share of the item: tpw tiles from K tile Q0 of 16 rows (tiles tix0.. of every
+        // plane chunk). Gate/up: warp -> matrix m (warps 0-7 gate, 8-15 up) and K part kp (of 8) of
+        // the item's 16 rows (a plane chunk holds [gate rows | up rows] of one plane); down: warp ->
+        // strip sb (of 8 x 16 rows) and K part kp (of 2). Both kinds share one decode call per
+        // fragment source, so that the decode code of a depth exists once.
+        const bool up = d.kind == 0;
+        const int m = up ? warp >> 3 : 2, sb = up ? 0 : warp >> 1, kp = up ? (warp & 7) : (warp & 1);
+        const int tpw = up ? (H / 128) / 8 : (I / 128) / 2, Q0 = kp * tpw;
+        const int tix0 = (up ? m * (H / 128) : sb * (I / 128)) + Q0;
+        const int ngr = (up ? H : I) / G;
+        if (!up && !fast && lane == 0) {
+            while (pipe::ld_acquire(&W.readyB[d.u]) < I / 128) {
+                if (pipe::globaltimer() > deadline) {
+                    fine = false;
+                    break;
+                }
+                __nanosleep(256);
+            }
+        }
+        fine = __shfl_sync(0xffffffffu, (int)fine, 0) != 0;
+        __syncwarp();
+        const unsigned char *pp[8];
 #pragma unroll
-            for (int p = 0; p < 8; ++p) {
-                const int cc = d.c0 + p;
-                pp[p] = S.ring[cc % NSLOT] + tix0 * 256 + lane * 8;
+        for (int p = 0; p < 8; ++p)
+            pp[p] = S.ring[(d.c0 + p) % NSLOT] + tix0 * 256 + lane * 8;
+        // meta chunk: scale rows (gate/up [16 gate | 16 up] rows, down 128 rows) x ngr groups, then the
+        // table heads (gate/up: gate and up per block; down: one per block), then (down items of one
+        // block) the members' h fragments and exponents
+        const float *sc0 = reinterpret_cast<const float *>(meta) + (up ? m * 16 + g : 16 * sb + g) * ngr + Q0 * (128 / G);
+        const float *sc1 = sc0 + 8 * ngr;
+        const unsigned char *tab0 = meta + (up ? 2 * 16 : 128) * ngr * 4;
+        for (int bi = 0; bi < nblk; ++bi) {
+            const int blk = blk0 + bi;
+            const int dd = V.bdepth(blk), nmem = V.bnmem(blk);
+            // B column g = 4*c + part: byte part of token c (part 3 and absent tokens: zero);
+            // lane t accumulates token t/2 (xfrag.cuh, dev::combine24)
+            const int c = g >> 2, part = g & 3, me = t >> 1;
+            const bool has = c < nmem && part < 3;
+            float acc0 = 0.0f, acc1 = 0.0f;
+            const unsigned char *tabs = tab0 + (up ? bi * 2 + m : bi) * TAB_BYTES;
+            const uint32_t *big = W.tabs + ((int64_t)blk * 3 + m) * kTabWords + 16;
+            const uint32_t *fptr = nullptr;
+            const int *exps = nullptr;
+            int fstep = KFW, fm;
+            if (up && stage_x) {
+                fm = 0;
+                fptr = has ? S.xs + Q0 * 4 * KFW + dev::frag_offset(part, t) : S.zeros;
+                fstep = has ? KFW : 0;
+                if (me < nmem)
+                    exps = S.xse;
+            } else if (up) {
+                fm = 1;
+                if (has)
+                    fptr = W.xfrag + ((int64_t)(V.bpair(blk, c) / k) * (H / 32) + Q0 * 4) * KFW + dev::frag_offset(part, t);
+                if (me < nmem)
+                    exps = W.xexp + (int64_t)(V.bpair(blk, me) / k) * (H / 128);
+            } else if (fast) {
+                // h fragments and exponents of the members arrived with the meta chunk
+                fm = 0;
+                const uint32_t *hf = reinterpret_cast<const uint32_t *>(tab0 + TAB_BYTES);
+                const int *he = reinterpret_cast<const int *>(hf + nmem * (I / 32) * KFW);
+                fptr = has ? hf + ((int64_t)c * (I / 32) + Q0 * 4) * KFW + dev::frag_offset(part, t) : S.zeros;
+                fstep = has ? KFW : 0;
+                if (me < nmem)
+                    exps = he + me * hexp_stride(I);
+            } else {
+                fm = 2;
+                if (has)
+                    fptr = W.hfrag + ((int64_t)V.bpair(blk, c) * (I / 32) + Q0 * 4) * KFW + dev::frag_offset(part, t);
+                if (me < nmem)
+                    exps = W.hexp + (int64_t)V.bpair(blk, me) * hexp_stride(I);
             }
-            {
-                const float *sc0 = reinterpret_cast<const float *>(meta) + (m * 16 + g) * ngr + Q0 * (128 / G);
-                const float *sc1 = sc0 + 8 * ngr;
-                for (int bi = 0; bi < nblk; ++bi) {
-                    const int blk = blk0 + bi;
-                    const int dd = V.bdepth(blk), nmem = V.bnmem(blk);
-                    // B column g = 4*c + part: byte part of token c (part 3 and absent tokens: zero);
-                    // lane t accumulates token t/2 (xfrag.cuh, dev::combine24)
-                    const int c = g >> 2, part = g & 3, me = t >> 1;
-                    const bool has = c < nmem && part < 3;
-                    float acc0 = 0.0f, acc1 = 0.0f;
-                    const int *exps = nullptr;
-                    if (me < nmem) {
-                        const int tok = V.bpair(blk, me) / k;
-                        exps = stage_x ? S.xse : W.xexp + (int64_t)tok * (H / 128);
-                    }
-                    const unsigned char *tabs = meta + 2 * 16 * ngr * 4 + (bi * 2 + m) * TAB_BYTES;
-                    const uint32_t *big = W.tabs + ((int64_t)blk * 3 + m) * kTabWords + 16;
-                    if (stage_x) {
-                        const uint32_t *fptr = has ? S.xs + Q0 * 4 * KFW + dev::frag_offset(part, t) : S.zeros;
-                        warp_block_any<GS, 0>(dd, pp, tpw, Q0, tabs, big, fptr, has ? KFW : 0, exps, sc0, sc1, acc0,
-                                              acc1);
-                    } else {
-                        const uint32_t *fptr = nullptr;
-                        if (has) {
-                            const int tok = V.bpair(blk, c) / k;
-                            fptr = W.xfrag + ((int64_t)tok * (H / 32) + Q0 * 4) * KFW + dev::frag_offset(part, t);
-                        }
-                        warp_block_any<GS, 1>(dd, pp, tpw, Q0, tabs, big, fptr, KFW, exps, sc0, sc1, acc0, acc1);
-                    }
-                    if ((t & 1) == 0 && me < nmem) {
-                        if (fast) {
-                            red[g * 4 + me] = acc0;
-                            red[(g + 8) * 4 + me] = acc1;
-                        } else {
-                            const int pair = V.bpair(blk, me);
-                            float *dst = W.pA + (((int64_t)pair * (I / 16) + d.strip) * 8 + kp) * 32 + m * 16;
-                            __stcg(dst + g, acc0);
-                            __stcg(dst + g + 8, acc1);
-                        }
-                    }
-                }
-            }
-            __syncwarp();
-            int last = 0;
-            if (fast) {
-                // the epilogue warp reduces the partials; the last warp only hands the item over
-                if (lane == 0) {
-                    __threadfence_block();
-                    if (atomicAdd(&S.cnt[qs], 1) == NCW - 1) {
-                        S.cnt[qs] = 0;
-                        pipe::mbar_arrive(&S.epi[qs]);
-                    }
-                }
-            } else if (lane == 0) {
-                last = (atom_add_acq_rel(&W.cntA[d.u * SA + d.strip], 1) == NCW - 1);
-            }
-            last = __shfl_sync(0xffffffffu, last, 0);
-            __syncwarp();
-            if (last) {
-                // h rows of the item: lanes 0-15 = row, every member of every block
-                for (int bi = 0; bi < nblk; ++bi) {
-                    const int blk = blk0 + bi, nmem = V.bnmem(blk);
-                    for (int c = 0; c < nmem; ++c) {
-                        const int pair = V.bpair(blk, c);
-                        const int rr = lane & 15;
-                        float gv = 0.0f, uv = 0.0f;
-                        const float *src = W.pA + (((int64_t)pair * (I / 16) + d.strip) * 8) * 32;
-#pragma unroll
-                        for (int kq = 0; kq < 8; ++kq) {
-                            gv += __ldcg(src + kq * 32 + rr);
-                            uv += __ldcg(src + kq * 32 + 16 + rr);
-                        }
-                        if (lane < 16)
-                            __stcg(W.h + (int64_t)pair * I + 16 * d.strip + rr, gv / (1.0f + expf(-gv)) * uv);
-                    }
-                }
-                gateup_tile_done(W, V, I, d.u, d.strip, blk0, nblk);
-            }
-        } else {
-            // down: warp -> strip sb (of 8 x 16 rows) and K part kp (of 2)
-            const int sb = warp >> 1, kp = warp & 1, tpw = (I / 128) / 2, Q0 = kp * tpw;
-            const int tix0 = sb * (I / 128) + Q0;
-            const int ngr = I / G;
-            if (!fast && lane == 0) {
-                while (pipe::ld_acquire(&W.readyB[d.u]) < I / 128) {
-                    if (pipe::globaltimer() > deadline) {
-                        fine = false;
-                        break;
-                    }
-                    __nanosleep(256);
-                }
-            }
-            fine = __shfl_sync(0xffffffffu, (int)fine, 0) != 0;
-            __syncwarp();
-            const unsigned char *pp[8];
-#pragma unroll
-            for (int p = 0; p < 8; ++p) {
-                const int cc = d.c0 + p;
-                pp[p] = S.ring[cc % NSLOT] + tix0 * 256 + lane * 8;
-            }
-            const float *sc0 = reinterpret_cast<const float *>(meta) + (16 * sb + g) * ngr + Q0 * (128 / G);
-            const float *sc1 = sc0 + 8 * ngr;
-            for (int bi = 0; bi < nblk; ++bi) {
-                const int blk = blk0 + bi;
-                const int dd = V.bdepth(blk), nmem = V.bnmem(blk);
-                const int c = g >> 2, part = g & 3, me = t >> 1;
-                const bool has = c < nmem && part < 3;
-                float acc0 = 0.0f, acc1 = 0.0f;
-                const unsigned char *tabs = meta + 128 * ngr * 4 + bi * TAB_BYTES;
-                const uint32_t *big = W.tabs + ((int64_t)blk * 3 + 2) * kTabWords + 16;
+            if (fm == 0)
+                warp_block_any<GS, 0>(dd, pp, tpw, Q0, tabs, big, fptr, fstep, exps, sc0, sc1, acc0, acc1);
+            else if (fm == 1)
+                warp_block_any<GS, 1>(dd, pp, tpw, Q0, tabs, big, fptr, fstep, exps, sc0, sc1, acc0, acc1);
+            else
+                warp_block_any<GS, 2>(dd, pp, tpw, Q0, tabs, big, fptr, fstep, exps, sc0, sc1, acc0, acc1);
+            if ((t & 1) == 0 && me < nmem) {
                 if (fast) {
-                    // h fragments and exponents of the members arrived with the meta chunk
-                    const uint32_t *hf = reinterpret_cast<const uint32_t *>(meta + 128 * ngr * 4 + TAB_BYTES);
-                    const int *he = reinterpret_cast<const int *>(hf + nmem * (I / 32) * KFW);
-                    const uint32_t *fptr =
-                        has ? hf + ((int64_t)c * (I / 32) + Q0 * 4) * KFW + dev::frag_offset(part, t) : S.zeros;
-                    const int *exps = (me < nmem) ? he + me * hexp_stride(I) : nullptr;
-                    warp_block_any<GS, 0>(dd, pp, tpw, Q0, tabs, big, fptr, has ? KFW : 0, exps, sc0, sc1, acc0,
-                                          acc1);
+                    red[g * 4 + me] = acc0;
+                    red[(g + 8) * 4 + me] = acc1;
                 } else {
-                    const uint32_t *fptr = nullptr;
-                    if (has) {
-                        const int pair = V.bpair(blk, c);
-                        fptr = W.hfrag + ((int64_t)pair * (I / 32) + Q0 * 4) * KFW + dev::frag_offset(part, t);
-                    }
-                    const int *exps = nullptr;
-                    if (me < nmem)
-                        exps = W.hexp + (int64_t)V.bpair(blk, me) * hexp_stride(I);
-                    warp_block_any<GS, 2>(dd, pp, tpw, Q0, tabs, big, fptr, KFW, exps, sc0, sc1, acc0, acc1);
+                    const int pair = V.bpair(blk, me);
+                    float *dst = up ? W.pA + (((int64_t)pair * (I / 16) + d.strip) * 8 + kp) * 32 + m * 16
+                                    : W.pB + (((int64_t)pair * (H / 16) + 8 * d.strip + sb) * 2 + kp) * 16;
+                    __stcg(dst + g, acc0);
+                    __stcg(dst + g + 8, acc1);
                 }
-                if ((t & 1) == 0 && me < nmem) {
-                    if (fast) {
-                        red[g * 4 + me] = acc0;
-                        red[(g + 8) * 4 + me] = acc1;
-                    } else {
-                        const int pair = V.bpair(blk, me);
-                        float *dst = W.pB + (((int64_t)pair * (H / 16) + 8 * d.strip + sb) * 2 + kp) * 16;
-                        __stcg(dst + g, acc0);
-                        __stcg(dst + g + 8, acc1);
+            }
+        }
+        __syncwarp();
+        int last = 0;
+        if (fast) {
+            // the epilogue warp reduces the partials; the last warp only hands the item over
+            if (lane == 0) {
+                __threadfence_block();
+                if (atomicAdd(&S.cnt[qs], 1) == NCW - 1) {
+                    S.cnt[qs] = 0;
+                    pipe::mbar_arrive(&S.epi[qs]);
+                }
+            }
+        } else if (lane == 0) {
+            last = (atom_add_acq_rel(up ? &W.cntA[d.u * SA + d.strip] : &W.cntB[d.u * SB + d.strip], 1) == NCW - 1);
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        __syncwarp();
+        if (last && up) {
+            // h rows of the item: lanes 0-15 = row, every member of every block
+            for (int bi = 0; bi < nblk; ++bi) {
+                const int blk = blk0 + bi, nmem = V.bnmem(blk);
+                for (int c = 0; c < nmem; ++c) {
+                    const int pair = V.bpair(blk, c);
+                    const int rr = lane & 15;
+                    float gv = 0.0f, uv = 0.0f;
+                    const float *src = W.pA + (((int64_t)pair * (I / 16) + d.strip) * 8) * 32;
+#pragma unroll
+                    for (int kq = 0; kq < 8; ++kq) {
+                        gv += __ldcg(src + kq * 32 + rr);
+                        uv += __ldcg(src + kq * 32 + 16 + rr);
+                    }
+                    if (lane < 16)
+                        __stcg(W.h + (int64_t)pair * I + 16 * d.strip + rr, gv / (1.0f + expf(-gv)) * uv);
+                }
+            }
+            gateup_tile_done(W, V, I, d.u, d.strip, blk0, nblk);
+        } else if (last) {
+            for (int bi = 0; bi < nblk; ++bi) {
+                const int blk = blk0 + bi, nmem = V.bnmem(blk);
+                for (int c = 0; c < nmem; ++c) {
+                    const int pair = V.bpair(blk, c);
+                    for (int r = lane; r < 128; r += 32) {
+                        const int s8 = r >> 4, rr = r & 15;
+                        const float *src = W.pB + (((int64_t)pair * (H / 16) + 8 * d.strip + s8) * 2) * 16;
+                        __stcg(W.part + (int64_t)pair * H + 128 * d.strip + r, __ldcg(src + rr) + __ldcg(src + 16 + rr));
                     }
                 }
             }
-            __syncwarp();
-            int last = 0;
-            if (fast) {
-                if (lane == 0) {
-                    __threadfence_block();
-                    if (atomicAdd(&S.cnt[qs], 1) == NCW - 1) {
-                        S.cnt[qs] = 0;
-                        pipe::mbar_arrive(&S.epi[qs]);
-                    }
-                }
-            } else if (lane == 0) {
-                last = (atom_add_acq_rel(&W.cntB[d.u * SB + d.strip], 1) == NCW - 1);
-            }
-            last = __shfl_sync(0xffffffffu, last, 0);
-            __syncwarp();
-            if (last) {
-                for (int bi = 0; bi < nblk; ++bi) {
-                    const int blk = blk0 + bi, nmem = V.bnmem(blk);
-                    for (int c = 0; c < nmem; ++c) {
-                        const int pair = V.bpair(blk, c);
-                        for (int r = lane; r < 128; r += 32) {
-                            const int s8 = r >> 4, rr = r & 15;
-                            const float *src = W.pB + (((int64_t)pair * (H / 16) + 8 * d.strip + s8) * 2) * 16;
-                            __stcg(W.part + (int64_t)pair * H + 128 * d.strip + r, __ldcg(src + rr) + __ldcg(src + 16 + rr));
-                        }
-                    }
-                }
-                for (int bi = 0; bi < nblk; ++bi) {
-                    const int blk = blk0 + bi, nmem = V.bnmem(blk);
-                    for (int c = 0; c < nmem; ++c)
-                        down_rows_done(a, V.bpair(blk, c), d.strip);
-                }
+            for (int bi = 0; bi < nblk; ++bi) {
+                const int blk = blk0 + bi, nmem = V.bnmem(blk);
+                for (int c = 0; c < nmem; ++c)
+                    down_rows_done(a, V.bpair(blk, c), d.strip);
             }
         }
         __syncwarp();
