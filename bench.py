@@ -54,6 +54,8 @@ def parse():
     # the stacked-layer decode through the HBM prefix cache (pinned host planes, side-stream top-ups)
     ap.add_argument("--workload", default="layer", choices=["layer", "cache", "batch"])
     ap.add_argument("--batch", type=int, default=32)
+    # batched decode: pairs an expert needs (at depth <= 4) to go to the tensor-core units
+    ap.add_argument("--tc-min", type=int, default=8)
     ap.add_argument("--layers", type=int, default=16)
     ap.add_argument("--cache-tokens", type=int, default=256)
     ap.add_argument("--cache-frac", type=float, default=0.4)
@@ -444,6 +446,7 @@ def batch_bench(args):
     import synth
     from bitplane_mixed_precision_b200.store import ResidentLayer
 
+    pm.set_tc_min_tokens(args.tc_min)
     Tb, nb = args.batch, 64
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
@@ -504,7 +507,7 @@ def batch_bench(args):
         per_exp.append(Tb * K_TOP / len(bmax))
     achieved = float(sum(alg) / sum(kdur)) / 1e9
     pk, pk_kind = peaks()
-    # tensor-core units of each batch (experts with >= 8 pairs at depth <= 4, units of <= 64 pairs):
+    # tensor-core units of each batch (experts with >= tc_min pairs at depth <= 4, units of <= 64 pairs):
     # counted by the library, and their MMA work (2 parts x levels x 2 flop per weight and token)
     tc_units, tc_rows, tc_pairs, tc_flop = [], [], [], []
     for b in range(nb):
@@ -516,7 +519,7 @@ def batch_bench(args):
         for e in np.unique(ids_h[b]):
             sel = (ids_h[b] == e) & (dep_h[b] <= 4)
             n = int(sel.sum())
-            if n < 8:
+            if n < args.tc_min:
                 continue
             pairs += n
             d = np.sort(dep_h[b][sel])[::-1]
@@ -566,7 +569,7 @@ def batch_bench(args):
     try:
         t_nt, _ = timed_steps()
     finally:
-        pm.set_tc_min_tokens(8)
+        pm.set_tc_min_tokens(args.tc_min)
     line = {
         "metric": f"batched MoE-layer decode tokens/s ({Tb} tokens per step)", "value": steps * Tb / t,
         "unit": "tokens/s", "n_gpus": 1, "steps": steps, "warmup": max(args.warmup, nb),
@@ -581,7 +584,8 @@ def batch_bench(args):
                      "kernel": "tensor-core kernels + moe_main_kernel (gate/up+SwiGLU, down, combine)",
                      "peak_kind": f"{pk_kind} hbm_gbs"},
         "expert_kernels_us": 1e6 * sum(kdur) / nb,
-        "tensor_core": {"units": float(np.mean(tc_units)), "operand_rows": float(np.mean(tc_rows)),
+        "tensor_core": {"min_pairs": args.tc_min, "units": float(np.mean(tc_units)),
+                        "operand_rows": float(np.mean(tc_rows)),
                         "pairs": float(np.mean(tc_pairs)), "pairs_frac": float(np.mean(tc_pairs)) / (Tb * K_TOP),
                         "mma_gflop_per_batch": float(np.mean(tc_flop)) / 1e9},
         "persistent_only": {"tokens_per_s": steps * Tb / t_nt, "ms_per_step": t_nt * 1e3 / steps},

@@ -90,7 +90,7 @@ def test_tensor_core_settings_are_checked_on_the_host(pm):
         with pytest.raises(pm.PmoeError) as ei:
             pm.set_tc_min_tokens(bad)
         assert ei.value.code == 1
-    for good in (0, 8, 16, 8):
+    for good in (0, 12, 16, 8):
         pm.set_tc_min_tokens(good)
     a = np.zeros((128, 128), np.int16)
     d = np.zeros((128, 64), np.float32)

@@ -125,24 +125,28 @@ def test_host_buffer_decode_step_matches_device_buffers(pm, T, k):
     R = ResidentLayer(E, H, I, G, device_fill(seed))
     sens = synth.sensitivities(seed, 0, E)
     logits, xb = tokens(seed, T, E, H)
-    y_dev, _, _, _ = run_step(pm, R, logits, xb, sens, k, 2.5)
-    nb = pm.decode_host_workspace_bytes(T, k, E, H, I)
-    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
-    d_sens = torch.from_numpy(sens).cuda()
-    lg = torch.from_numpy(logits).pin_memory()
-    x = torch.from_numpy(xb.view(np.int16)).pin_memory()
-    y = torch.full((T * H,), float("nan"), dtype=torch.float32).pin_memory()
-    pm.moe_decode_step_host(R.layer, lg, d_sens, x, T, k, 2.5, y, ws, nb)
-    torch.cuda.synchronize()
-    assert pm.layer_error(ws) == (0, 0)
-    np.testing.assert_array_equal(y.numpy().reshape(T, H), y_dev)
-    if T >= 24:
-        assert pm.layer_counts(ws)[2] > 0  # tensor-core units were formed
-    y_np = np.full(T * H, np.nan, np.float32)
-    pm.moe_decode_step_host(R.layer, np.ascontiguousarray(logits), d_sens, xb.view(np.int16).copy(), T, k, 2.5,
-                            y_np, ws, nb)
-    torch.cuda.synchronize()
-    np.testing.assert_array_equal(y_np.reshape(T, H), y_dev)
+    pm.set_tc_min_tokens(8)  # (the default) tensor-core units from 8 pairs
+    try:
+        y_dev, _, _, _ = run_step(pm, R, logits, xb, sens, k, 2.5)
+        nb = pm.decode_host_workspace_bytes(T, k, E, H, I)
+        ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+        d_sens = torch.from_numpy(sens).cuda()
+        lg = torch.from_numpy(logits).pin_memory()
+        x = torch.from_numpy(xb.view(np.int16)).pin_memory()
+        y = torch.full((T * H,), float("nan"), dtype=torch.float32).pin_memory()
+        pm.moe_decode_step_host(R.layer, lg, d_sens, x, T, k, 2.5, y, ws, nb)
+        torch.cuda.synchronize()
+        assert pm.layer_error(ws) == (0, 0)
+        np.testing.assert_array_equal(y.numpy().reshape(T, H), y_dev)
+        if T >= 24:
+            assert pm.layer_counts(ws)[2] > 0  # tensor-core units were formed
+        y_np = np.full(T * H, np.nan, np.float32)
+        pm.moe_decode_step_host(R.layer, np.ascontiguousarray(logits), d_sens, xb.view(np.int16).copy(), T, k, 2.5,
+                                y_np, ws, nb)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(y_np.reshape(T, H), y_dev)
+    finally:
+        pm.set_tc_min_tokens(8)
 
 
 def test_zero_tokens_is_a_no_op(pm):

@@ -23,6 +23,7 @@ pytestmark = pytest.mark.gpu
 
 E, H, I, G = 16, 1024, 256, 128
 SEED = 2031
+TC_DEFAULT = 8  # the library's default threshold (pairs per expert)
 
 
 @pytest.fixture(scope="module")
@@ -75,24 +76,29 @@ def _batch(T, k, rng):
     return ids, w, dep, x
 
 
-@pytest.mark.parametrize("T", [24, 128])
-def test_layer_with_tensor_core_units(pm, mid, T):
+@pytest.mark.parametrize("T,tc_min", [(24, 8), (128, 8), (128, 12)])
+def test_layer_with_tensor_core_units(pm, mid, T, tc_min):
+    """The rule at the default threshold (8 pairs, the smallest the workspace allows) and at 12."""
     R, O = mid
     k = 4
     ids, w, dep, x = _batch(T, k, np.random.default_rng(T))
     y = torch.empty(T * H, dtype=torch.float32, device="cuda")
     nb = pm.layer_workspace_bytes(T, k, E, H, I)
     ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
-    pm.moe_layer_fwd(R.layer, torch.from_numpy(x.view(np.int16)).cuda(), torch.from_numpy(ids).cuda(),
-                     torch.from_numpy(w).cuda(), torch.from_numpy(dep).cuda(), T, k, y, ws, nb)
-    torch.cuda.synchronize()
+    pm.set_tc_min_tokens(tc_min)
+    try:
+        pm.moe_layer_fwd(R.layer, torch.from_numpy(x.view(np.int16)).cuda(), torch.from_numpy(ids).cuda(),
+                         torch.from_numpy(w).cuda(), torch.from_numpy(dep).cuda(), T, k, y, ws, nb)
+        torch.cuda.synchronize()
+    finally:
+        pm.set_tc_min_tokens(TC_DEFAULT)
     assert pm.layer_error(ws) == (0, 0)
     blocks, units, tcu, rows = pm.layer_counts(ws)
-    # every expert with at least 8 pairs at depth <= 4 gives them to units of at most 64 pairs
+    # every expert with at least tc_min pairs at depth <= 4 gives them to units of at most 64 pairs
     shallow = np.bincount(ids[dep <= 4], minlength=E)
-    expect = sum((int(n) + 63) // 64 for n in shallow if n >= 8)
+    expect = sum((int(n) + 63) // 64 for n in shallow if n >= tc_min)
     assert tcu == expect >= 3, (tcu, expect)
-    assert rows >= int(shallow[shallow >= 8].sum()) and rows % 16 == 0
+    assert rows >= int(shallow[shallow >= tc_min].sum()) and rows % 16 == 0
     ref = O.run(E, ids, w, dep, synth.bf16_to_f32(x).astype(np.float64))
     got = y.cpu().numpy().reshape(T, H)
     for t in range(T):
