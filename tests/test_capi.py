@@ -134,6 +134,8 @@ def test_host_buffer_decode_step_is_checked_on_the_host(pm):
     with pytest.raises(pm.PmoeError) as ei:
         pm.moe_decode_step_host(L, host, 0x500000, host, T, k, 2.5, host, 0x600000, need - 256)
     assert ei.value.code == 5
+    # zero tokens: nothing to do, no buffer is touched (all may be null)
+    pm.moe_decode_step_host(L, None, None, None, 0, k, 2.5, None, None, 0)
 
 
 def test_cache_aware_select_matches_oracle(pm, oracle_mod):
