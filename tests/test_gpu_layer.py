@@ -111,8 +111,11 @@ def test_uniform_depth_layer(pm, b):
         assert_close(got[t], ref[t], msg=f"b={b} token {t}")
 
 
-def test_group_size_64(pm):
-    check_layer(pm, 42, 16, 1024, 512, 64, 4, 3)
+@pytest.mark.parametrize("G,T", [(64, 3), (32, 1), (32, 3)])
+def test_group_sizes_64_and_32(pm, G, T):
+    """Scale groups of 64 and 32 columns (two and four groups per 128-column tile), batch 1 and a
+    3-token batch."""
+    check_layer(pm, 42, 16, 1024, 512, G, 4, T)
 
 
 @pytest.mark.parametrize("T,k", [(1, 4), (3, 4), (24, 10)])
