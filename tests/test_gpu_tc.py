@@ -105,6 +105,28 @@ def test_layer_with_tensor_core_units(pm, mid, T, tc_min):
         assert_close(got[t], ref[t], msg=f"token {t}")
 
 
+@pytest.mark.parametrize("Gs", [64, 32])
+def test_tensor_core_units_with_smaller_scale_groups(pm, Gs):
+    """Scale groups of 64 and 32 columns: the epilogue applies two or four group scales per 128-column
+    tile of the tensor-core accumulators; every token against the oracle."""
+    R = ResidentLayer(E, H, I, Gs, device_fill(SEED + Gs))
+    O = OracleExperts(SEED + Gs, H, I, Gs)
+    T, k = 24, 4
+    ids, w, dep, x = _batch(T, k, np.random.default_rng(T))
+    y = torch.empty(T * H, dtype=torch.float32, device="cuda")
+    nb = pm.layer_workspace_bytes(T, k, E, H, I)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    pm.moe_layer_fwd(R.layer, torch.from_numpy(x.view(np.int16)).cuda(), torch.from_numpy(ids).cuda(),
+                     torch.from_numpy(w).cuda(), torch.from_numpy(dep).cuda(), T, k, y, ws, nb)
+    torch.cuda.synchronize()
+    assert pm.layer_error(ws) == (0, 0)
+    assert pm.layer_counts(ws)[2] >= 3  # tensor-core units were formed
+    ref = O.run(E, ids, w, dep, synth.bf16_to_f32(x).astype(np.float64))
+    got = y.cpu().numpy().reshape(T, H)
+    for t in range(T):
+        assert_close(got[t], ref[t], msg=f"G={Gs} token {t}")
+
+
 def test_small_batches_keep_the_persistent_path(pm, mid):
     """Fewer than 8 tokens (or no expert with 8 shallow pairs): no tensor-core unit."""
     R, O = mid
